@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the Gemma 3 5:1 block attention on B200.
+
+One step = one 5:1 block (five local layers, one global layer) of prefill on
+the 27B-shaped 8K-token workload, through g3attn_prefill.  The same run also
+times one decode block step on the 64-sequence, 4K-128K-token workload (six
+g3attn_decode calls) and reports it under "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl g3attn|reference]
+
+Under torchrun each rank runs the whole workload on its own GPU (the units
+are independent, no data-path collective): weak scaling, value = all ranks'
+FLOPs / the slowest rank's time.  `--impl reference` times the float64 CPU
+oracle on bounded samples of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import inputs  # noqa: E402
+from global_gqa_b200 import metrics  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s (unmasked FLOPs, 5:1 block) & decode KV GB/s, 1 B200"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "prefill_attention_traffic.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "sm100_ptx.cuh", "g3_internal.h"):
+        with open(os.path.join(ROOT, "global_gqa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------- clock sampler
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, torch_dev_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            h = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(torch_dev_index).uuid)
+                h = nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[torch_dev_index]) if vis and vis.split(",")[0].isdigit() else torch_dev_index
+                h = nv.nvmlDeviceGetHandleByIndex(idx)
+            self._h = h
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU baselines
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_prefill_sample(cfg, budget_s: float, seed: int = 0):
+    """Time the oracle on sampled query rows of every layer of the block.
+
+    Returns (flops, seconds, n_rows).  Rows come from a seeded permutation and
+    are processed in groups of 64 until the time budget is spent (at least one
+    group per layer).
+    """
+    from oracle import attention as O
+    blk = cfg.block()
+    rng = np.random.default_rng(seed)
+    flops, secs, nrows = 0.0, 0.0, 0
+    key = (cfg.name, len(blk))
+    if key not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS[key] = [inputs.config_layer_inputs(cfg, li) for li in range(len(blk))]
+    xs = _ORACLE_INPUTS[key]
+    order = rng.permutation(cfg.S)
+    g = 0
+    while True:
+        for li, L in enumerate(blk):
+            rows = np.sort(order[(g * 64) % cfg.S:(g * 64) % cfg.S + 64])
+            x = xs[li]
+            lo, hi = metrics.row_intervals(cfg.S, L.kind, L.window)
+            t0 = time.perf_counter()
+            O.prefill_rows(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind,
+                           L.window, L.rope_base, L.interp, x["spans"], rows=rows)
+            secs += time.perf_counter() - t0
+            flops += 4.0 * cfg.D * cfg.Hq * cfg.B * float(np.sum(hi[rows] - lo[rows] + 1))
+            nrows += rows.size
+        g += 1
+        if secs >= budget_s:
+            return flops, secs, nrows
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import global_gqa_b200 as g3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    g3.lib()
+    pk, pk_kind = peaks()
+    cfg = inputs.BLOCK_8K
+    blk = cfg.block()
+
+    # ---- prefill block inputs, resident in HBM (one set per layer)
+    layers = []
+    for li, L in enumerate(blk):
+        x = inputs.config_layer_inputs(cfg, li)
+        xd = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+        xd["out"] = torch.empty_like(xd["q"])
+        layers.append((L, xd))
+    ws = torch.empty(g3.prefill_workspace_size(cfg.B, cfg.S, cfg.Hq, cfg.Hkv, cfg.D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    block_flops = metrics.block_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, blk)
+
+    def prefill_step():
+        for L, x in layers:
+            g3.prefill(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind, L.window,
+                       L.rope_base, L.interp, x["spans"], out=x["out"], ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    if g3.check_device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    sampler = ClockSampler(local_rank)
+    g3.trace_collect()
+    barrier()
+    with sampler:
+        g3.trace_enable(True)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            prefill_step()
+        e1.record(stream)
+        barrier()
+        g3.trace_enable(False)
+    ms = e0.elapsed_time(e1)
+    trace = g3.trace_collect()
+    if g3.check_device_error(ws) != 0:
+        raise RuntimeError("device error in the timed region")
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = block_flops * args.steps * world / (ms_max * 1e-3) / 1e12
+
+    n_attn, attn_ms = trace.get("prefill_attention", (0, 0.0))
+    achieved = block_flops * args.steps / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
+    traffic = None
+    try:
+        with open(TRAFFIC_PATH) as f:
+            tr = json.load(f)
+        if tr.get("source_hash") == kernel_source_hash():
+            traffic = tr.get("bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    peak_tf = pk["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
+                "kernel": "prefill_attention", "peak_kind": f"{pk_kind} dense bf16 burst",
+                "launches": n_attn, "avg_launch_ms": attn_ms / max(n_attn, 1)}
+    kernels = {k: {"launches": v[0], "ms": v[1], "share": v[1] / max(sum(x[1] for x in trace.values()), 1e-9)}
+               for k, v in trace.items()}
+
+    # ---- end to end through the public API from pinned host memory
+    host = []
+    for L, x in layers:
+        hx = {k: (v.cpu().pin_memory() if v is not None and k != "out" else None) for k, v in x.items()}
+        hx["out"] = torch.empty(x["out"].shape, dtype=x["out"].dtype).pin_memory()
+        host.append((L, hx))
+    h2d = sum(v.numel() * v.element_size() for _, hx in host for k, v in hx.items() if v is not None and k != "out")
+    d2h = sum(hx["out"].numel() * hx["out"].element_size() for _, hx in host)
+
+    def e2e_step():
+        for (L, hx), (_, x) in zip(host, layers):
+            for k in ("q", "k", "v", "q_gamma", "k_gamma", "positions"):
+                x[k].copy_(hx[k], non_blocking=True)
+            g3.prefill(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind, L.window,
+                       L.rope_base, L.interp, x["spans"], out=x["out"], ws=ws, stream=stream)
+            hx["out"].copy_(x["out"], non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 20))
+    e2e_step()
+    barrier()
+    w0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    wall = time.perf_counter() - w0
+    e2e_ms = torch.tensor([max(e0.elapsed_time(e1), wall * 1e3)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = block_flops * e2e_steps * world / (float(e2e_ms.item()) * 1e-3) / 1e12
+    del host
+
+    # ---- decode block step on the 64 x (4K..128K) workload
+    decode = None
+    if not args.no_decode:
+        decode = run_decode(args, dev, stream, world, pk, pk_kind)
+
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.B, "seq_len": cfg.S, "q_heads": cfg.Hq, "kv_heads": cfg.Hkv,
+                   "head_dim": cfg.D, "block": "5 local (W=1024, base 1e4) + 1 global (base 1e6, interp 8)",
+                   "unmasked_flops_per_step": block_flops,
+                   "l2": "inputs larger than L2: each layer reads 128 MiB of q/k/v and writes 64 MiB",
+                   "parallelism": f"independent replicas x{world}"},
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": sum(v[0] for v in trace.values()),
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "decode": decode,
+    }
+    return line
+
+
+def run_decode(args, dev, stream, world, pk, pk_kind):
+    import torch
+    import global_gqa_b200 as g3
+    cfg = inputs.DECODE_B64
+    blk = cfg.block()
+    lens = inputs.decode_lengths(cfg.B, cfg.len_lo, cfg.len_hi, cfg.seed)
+    sl = lens.to(dev)
+    caches = []
+    for li, L in enumerate(blk):
+        if L.kind == 0:
+            kc = torch.empty(cfg.B, cfg.Hkv, cfg.window, cfg.D, dtype=torch.bfloat16, device=dev)
+        else:
+            kc = torch.empty(cfg.B, cfg.Hkv, cfg.global_capacity, cfg.D, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        inputs.device_fill_normal_bf16(kc, inputs.seed_for(cfg.seed, li, inputs.T_KC))
+        inputs.device_fill_normal_bf16(vc, inputs.seed_for(cfg.seed, li, inputs.T_VC))
+        x = {k: v.to(dev) for k, v in inputs.decode_step_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, seed=cfg.seed,
+                                                               layer=li).items()}
+        x["out"] = torch.empty_like(x["q"])
+        caches.append((L, kc, vc, x))
+    ws = torch.empty(g3.decode_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.len_hi), dtype=torch.uint8,
+                     device=dev)
+    step_bytes = sum(metrics.decode_kv_bytes(lens.numpy(), cfg.Hkv, cfg.D, L.kind, L.window) for L in blk)
+
+    def step():
+        for L, kc, vc, x in caches:
+            g3.decode(x["q"], x["k_new"], x["v_new"], x["q_gamma"], x["k_gamma"], kc, vc, sl, cfg.len_hi, L.kind,
+                      L.window, L.rope_base, L.interp, out=x["out"], ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if g3.check_device_error(ws) != 0:
+        raise RuntimeError("device error in decode warm-up")
+    g3.trace_collect()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    g3.trace_enable(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    g3.trace_enable(False)
+    if world > 1:
+        torch.distributed.barrier()
+    trace = g3.trace_collect()
+    ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
+    ms = float(ms.item())
+    gbs = step_bytes * args.steps * world / (ms * 1e-3) / 1e9
+    n_split, split_ms = trace.get("decode_split", (0, 0.0))
+    ach = step_bytes * args.steps / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
+    del caches
+    torch.cuda.empty_cache()
+    return {
+        "metric": "decode KV GB/s (5:1 block)", "value": gbs, "unit": "GB/s", "ms_per_step": ms / args.steps,
+        "config": {"workload": cfg.name, "batch": cfg.B, "context": f"U[{cfg.len_lo},{cfg.len_hi}]",
+                   "kv_bytes_per_step": step_bytes, "l2": "inputs larger than L2 (~38 GB of cache read per step)"},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": (ach / pk["hbm_gbs"]) if ach else None, "traffic": None, "kernel": "decode_split",
+                     "peak_kind": f"{pk_kind} copy bandwidth", "launches": n_split},
+        "kernels": {k: {"launches": v[0], "ms": v[1]} for k, v in trace.items()},
+        "gpu_launches": sum(v[0] for v in trace.values()),
+    }
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args):
+    cfg = inputs.BLOCK_8K
+    cores = blas_threads()
+    for _ in range(args.warmup):
+        oracle_prefill_sample(cfg, 0.0, seed=1)
+    flops, secs, rows = 0.0, 0.0, 0
+    for s in range(args.steps):
+        f, t, r = oracle_prefill_sample(cfg, 0.0, seed=100 + s)
+        flops, secs, rows = flops + f, secs + t, rows + r
+    value = flops / secs / 1e12
+    sample = f"{rows} query rows (64 per layer per step, all 32 heads) of the {cfg.name} block"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.B, "seq_len": cfg.S, "q_heads": cfg.Hq,
+                       "kv_heads": cfg.Hkv, "head_dim": cfg.D},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="g3attn", choices=["g3attn", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local_rank))
+    line = run_gpu(args, rank, world, local_rank)
+    if rank == 0 and world == 1:
+        f, s, r = oracle_prefill_sample(inputs.BLOCK_8K, args.cpu_budget)
+        line["cpu_baseline"] = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "seconds": s,
+                                "sample": f"{r} query rows (groups of 64 per layer, all 32 heads) of the "
+                                          f"{inputs.BLOCK_8K.name} block, float64 numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

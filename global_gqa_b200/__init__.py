@@ -1,0 +1,227 @@
+"""Python binding of libg3attn (Gemma 3 5:1 block attention on B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library behind the C ABI declared in include/g3attn.h.  torch supplies device
+memory and the current stream.  There is no fallback: if the library is not
+built or no CUDA device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Tuple
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB_PATH = os.path.join(HERE, "libg3attn.so")
+HEADER_PATH = os.path.join(ROOT, "include", "g3attn.h")
+
+LOCAL = 0
+GLOBAL = 1
+
+STATUS = {0: "G3_OK", 1: "G3_ERR_INVALID_ARG", 2: "G3_ERR_UNSUPPORTED", 3: "G3_ERR_WORKSPACE",
+          4: "G3_ERR_CUDA", 5: "G3_ERR_TIMEOUT"}
+
+
+class G3Error(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {detail}")
+
+
+class KernelTrace(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64), ("total_ms", ctypes.c_double)]
+
+
+_lib = None
+
+_vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+
+_SIGS = {
+    "g3attn_prefill_workspace_size": (_sz, [_i32] * 5),
+    "g3attn_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _i32, _f32, _f32, _vp, _i32,
+                                      _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "g3attn_decode_workspace_size": (_sz, [_i32] * 5),
+    "g3attn_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, ctypes.c_int, _i32,
+                                     _f32, _f32, _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
+    "g3attn_check_device_error": (ctypes.c_int, [_vp, _vp]),
+    "g3attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "g3attn_last_error": (ctypes.c_char_p, []),
+    "g3attn_trace_enable": (ctypes.c_int, [ctypes.c_int]),
+    "g3attn_trace_collect": (_i32, [ctypes.POINTER(KernelTrace), _i32]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m global_gqa_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/g3attn.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(g3attn_\w+)\s*\(", text)))
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        detail = lib().g3attn_last_error().decode(errors="replace")
+        raise G3Error(status, where, detail)
+
+
+def prefill_workspace_size(B: int, S: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().g3attn_prefill_workspace_size(B, S, Hq, Hkv, D))
+
+
+def decode_workspace_size(B: int, Hq: int, Hkv: int, D: int, max_seq_len: int) -> int:
+    return int(lib().g3attn_decode_workspace_size(B, Hq, Hkv, D, max_seq_len))
+
+
+# ----------------------------------------------------------- torch plumbing
+def _torch():
+    import torch
+    return torch
+
+
+_workspaces = {}
+
+
+def workspace(nbytes: int, device, tag: str = "default"):
+    """A cached uint8 device buffer of at least nbytes (256-byte aligned)."""
+    torch = _torch()
+    key = (str(device), tag)
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _workspaces[key] = buf
+    return buf
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream, device) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _req(t, name, dtype, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def prefill(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, window: int, rope_base: float,
+            interp_factor: float, image_spans=None, *, out=None, return_lse: bool = False,
+            k_cache=None, v_cache=None, ws=None, stream=None):
+    """One attention layer over full sequences; returns out (and lse).
+
+    q [B,S,Hq,D] bf16, k/v [B,S,Hkv,D] bf16 (raw projections), gammas fp32
+    [D], positions int32 [B,S], image_spans int32 [B,n,2] or None.
+    """
+    torch = _torch()
+    _req(q, "q", torch.bfloat16)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _req(k, "k", torch.bfloat16, (B, S, Hkv, D))
+    _req(v, "v", torch.bfloat16, (B, S, Hkv, D))
+    _req(q_gamma, "q_gamma", torch.float32, (D,))
+    _req(k_gamma, "k_gamma", torch.float32, (D,))
+    _req(positions, "positions", torch.int32, (B, S))
+    n_spans = 0
+    if image_spans is not None:
+        _req(image_spans, "image_spans", torch.int32)
+        if image_spans.dim() != 3 or image_spans.shape[0] != B or image_spans.shape[2] != 2:
+            raise ValueError("image_spans must be [B, n, 2]")
+        n_spans = int(image_spans.shape[1])
+        if n_spans == 0:
+            image_spans = None
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, S, dtype=torch.float32, device=q.device) if return_lse else None
+    cap = 0
+    if k_cache is not None:
+        _req(k_cache, "k_cache", torch.bfloat16)
+        _req(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+        cap = int(k_cache.shape[2])
+    need = prefill_workspace_size(B, S, Hq, Hkv, D)
+    wsb = ws if ws is not None else workspace(need, q.device)
+    st = lib().g3attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
+                              int(layer_kind), int(window), float(rope_base), float(interp_factor),
+                              _ptr(image_spans), n_spans, B, S, Hq, Hkv, D, _ptr(out), _ptr(lse),
+                              _ptr(k_cache), _ptr(v_cache), cap, wsb.data_ptr(), wsb.numel(),
+                              _stream_ptr(stream, q.device))
+    _check(st, "g3attn_prefill")
+    return (out, lse) if return_lse else out
+
+
+def decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, seq_lens, max_seq_len: int,
+           layer_kind: int, window: int, rope_base: float, interp_factor: float, *, out=None,
+           ws=None, stream=None):
+    """One decode step: writes the new token into the cache and returns out [B,Hq,D]."""
+    torch = _torch()
+    _req(q, "q", torch.bfloat16)
+    B, Hq, D = q.shape
+    Hkv = k_new.shape[1]
+    _req(k_new, "k_new", torch.bfloat16, (B, Hkv, D))
+    _req(v_new, "v_new", torch.bfloat16, (B, Hkv, D))
+    _req(q_gamma, "q_gamma", torch.float32, (D,))
+    _req(k_gamma, "k_gamma", torch.float32, (D,))
+    _req(k_cache, "k_cache", torch.bfloat16)
+    cap = int(k_cache.shape[2])
+    _req(k_cache, "k_cache", torch.bfloat16, (B, Hkv, cap, D))
+    _req(v_cache, "v_cache", torch.bfloat16, (B, Hkv, cap, D))
+    _req(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_size(B, Hq, Hkv, D, max_seq_len)
+    wsb = ws if ws is not None else workspace(need, q.device)
+    st = lib().g3attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_gamma), _ptr(k_gamma),
+                             _ptr(k_cache), _ptr(v_cache), cap, _ptr(seq_lens), int(max_seq_len),
+                             int(layer_kind), int(window), float(rope_base), float(interp_factor),
+                             B, Hq, Hkv, D, _ptr(out), wsb.data_ptr(), wsb.numel(),
+                             _stream_ptr(stream, q.device))
+    _check(st, "g3attn_decode")
+    return out
+
+
+def check_device_error(ws=None, device=None, stream=None) -> int:
+    """Status recorded on the device by the last call using this workspace."""
+    torch = _torch()
+    if ws is None:
+        dev = torch.device(device if device is not None else "cuda")
+        ws = workspace(256, dev)
+    return int(lib().g3attn_check_device_error(ws.data_ptr(), _stream_ptr(stream, ws.device)))
+
+
+def trace_enable(on: bool = True) -> None:
+    lib().g3attn_trace_enable(1 if on else 0)
+
+
+def trace_collect() -> dict:
+    arr = (KernelTrace * 32)()
+    n = lib().g3attn_trace_collect(arr, 32)
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}

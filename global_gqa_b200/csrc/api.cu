@@ -1,0 +1,407 @@
+// Host side of the C ABI declared in include/g3attn.h: argument validation,
+// workspace carving, TMA descriptor encoding, kernel launches and tracing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/g3attn.h"
+#include "g3_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+g3_status fail(g3_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+g3_status fail(g3_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ tracing
+struct TraceEntry {
+  std::string name;
+  cudaEvent_t start, stop;
+};
+struct TraceState {
+  std::mutex mu;
+  bool enabled = false;
+  std::vector<TraceEntry> pending;
+  std::vector<cudaEvent_t> pool;
+} g_trace;
+
+cudaEvent_t trace_event() {
+  if (!g_trace.pool.empty()) {
+    cudaEvent_t e = g_trace.pool.back();
+    g_trace.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Runs `launch` bracketed by trace events when tracing is on.
+template <class F>
+cudaError_t traced(const char* name, cudaStream_t st, F&& launch) {
+  if (!g_trace.enabled) return launch();
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  TraceEntry e{name, trace_event(), trace_event()};
+  cudaEventRecord(e.start, st);
+  cudaError_t r = launch();
+  cudaEventRecord(e.stop, st);
+  g_trace.pending.push_back(e);
+  return r;
+}
+
+// ------------------------------------------------------------ TMA encoding
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B, S, H, D] bf16, boxes of 64 features x 1 head x 128 tokens x 1 sequence,
+// 128-byte swizzle (matches the tcgen05 shared-memory descriptors).
+bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------- workspace maps
+struct PrefillWs {
+  size_t lo, hi, q_hat, k_hat, total;
+};
+bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w) {
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || D < 1) return false;
+  const size_t rows = (size_t)B * S;
+  size_t off = g3::kHeaderBytes;
+  w->lo = off;
+  off = align_up(off + rows * 4, 1024);
+  w->hi = off;
+  off = align_up(off + rows * 4, 1024);
+  w->q_hat = off;
+  off = align_up(off + rows * Hq * D * 2, 1024);
+  w->k_hat = off;
+  off = align_up(off + rows * Hkv * D * 2, 1024);
+  w->total = off;
+  return true;
+}
+
+struct DecodeWs {
+  size_t q_hat, n_slots, part_ml, part_o, total;
+  int n_chunks;
+};
+bool decode_ws(int B, int Hq, int Hkv, int D, int max_len, DecodeWs* w) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || max_len < 1) return false;
+  w->n_chunks = (max_len + g3::kDecodeChunk - 1) / g3::kDecodeChunk;
+  size_t off = g3::kHeaderBytes;
+  w->q_hat = off;
+  off = align_up(off + (size_t)B * Hq * D * 4, 256);
+  w->n_slots = off;
+  off = align_up(off + (size_t)B * 4, 256);
+  w->part_ml = off;
+  off = align_up(off + (size_t)B * Hq * w->n_chunks * 2 * 4, 256);
+  w->part_o = off;
+  off = align_up(off + (size_t)B * Hq * w->n_chunks * D * 4, 256);
+  w->total = off;
+  return true;
+}
+
+bool supported_d(int D) { return D == 64 || D == 128; }
+
+}  // namespace
+
+extern "C" {
+
+const char* g3attn_status_string(g3_status s) {
+  switch (s) {
+    case G3_OK: return "ok";
+    case G3_ERR_INVALID_ARG: return "invalid argument";
+    case G3_ERR_UNSUPPORTED: return "unsupported configuration";
+    case G3_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case G3_ERR_CUDA: return "CUDA error";
+    case G3_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* g3attn_last_error(void) { return g_last_error.c_str(); }
+
+size_t g3attn_prefill_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D) {
+  PrefillWs w;
+  if (!prefill_ws(B, S, Hq, Hkv, D, &w)) return 0;
+  return w.total;
+}
+
+size_t g3attn_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t max_seq_len) {
+  DecodeWs w;
+  if (!decode_ws(B, Hq, Hkv, D, max_seq_len, &w)) return 0;
+  return w.total;
+}
+
+g3_status g3attn_prefill(const void* q, const void* k, const void* v, const float* q_gamma, const float* k_gamma,
+                         const int32_t* positions, g3_layer_kind layer_kind, int32_t window, float rope_base,
+                         float interp_factor, const int32_t* image_spans, int32_t n_spans, int32_t B, int32_t S,
+                         int32_t Hq, int32_t Hkv, int32_t D, void* out, float* lse, void* k_cache, void* v_cache,
+                         int32_t cache_capacity, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !q_gamma || !k_gamma || !positions || !out)
+    return fail(G3_ERR_INVALID_ARG, "prefill: a required pointer is NULL");
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || D < 1)
+    return fail(G3_ERR_INVALID_ARG, "prefill: sizes must be positive (B=%d S=%d Hq=%d Hkv=%d D=%d)", B, S, Hq, Hkv, D);
+  if (Hq % Hkv != 0) return fail(G3_ERR_INVALID_ARG, "prefill: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
+  if (layer_kind != G3_LAYER_LOCAL && layer_kind != G3_LAYER_GLOBAL)
+    return fail(G3_ERR_INVALID_ARG, "prefill: bad layer kind %d", (int)layer_kind);
+  if (layer_kind == G3_LAYER_LOCAL && window < 1) return fail(G3_ERR_INVALID_ARG, "prefill: window < 1");
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return fail(G3_ERR_INVALID_ARG, "prefill: bad rope_base");
+  if (!(interp_factor > 0.f) || !std::isfinite(interp_factor))
+    return fail(G3_ERR_INVALID_ARG, "prefill: bad interp_factor");
+  if (n_spans < 0 || (n_spans > 0 && image_spans == nullptr) || (n_spans == 0 && image_spans != nullptr))
+    return fail(G3_ERR_INVALID_ARG, "prefill: image_spans must be NULL iff n_spans == 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(G3_ERR_INVALID_ARG, "prefill: q, k, v and out must be 16-byte aligned");
+  if ((k_cache == nullptr) != (v_cache == nullptr))
+    return fail(G3_ERR_INVALID_ARG, "prefill: give both caches or neither");
+  if (k_cache != nullptr) {
+    if (!aligned16(k_cache) || !aligned16(v_cache))
+      return fail(G3_ERR_INVALID_ARG, "prefill: caches must be 16-byte aligned");
+    if (layer_kind == G3_LAYER_GLOBAL && cache_capacity < S)
+      return fail(G3_ERR_INVALID_ARG, "prefill: global cache capacity %d < S %d", cache_capacity, S);
+    if (layer_kind == G3_LAYER_LOCAL && cache_capacity != window)
+      return fail(G3_ERR_INVALID_ARG, "prefill: local ring capacity %d != window %d", cache_capacity, window);
+  }
+  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "prefill: head_dim %d not built (64, 128)", D);
+  if ((size_t)B * S * Hq * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "prefill: problem too large");
+  const int G = Hq / Hkv;
+  const int hpc = (G % 2 == 0) ? 2 : 1;
+  const long long n_qtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
+  if (n_qtiles * B * Hkv * (G / hpc) > 0x7fffffffLL) return fail(G3_ERR_UNSUPPORTED, "prefill: grid too large");
+
+  PrefillWs w;
+  prefill_ws(B, S, Hq, Hkv, D, &w);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(G3_ERR_WORKSPACE, "prefill: workspace NULL or not 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(G3_ERR_WORKSPACE, "prefill: workspace %zu bytes < required %zu", workspace_bytes, w.total);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* err = reinterpret_cast<int*>(ws);
+
+  g3::PrologueParams pp{};
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.q_gamma = q_gamma;
+  pp.k_gamma = k_gamma;
+  pp.positions = positions;
+  pp.spans = image_spans;
+  pp.n_spans = n_spans;
+  pp.B = B;
+  pp.S = S;
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.kind = (int)layer_kind;
+  pp.window = layer_kind == G3_LAYER_LOCAL ? window : S;
+  pp.rope_base = rope_base;
+  pp.interp = interp_factor;
+  pp.q_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.q_hat);
+  pp.k_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.k_hat);
+  pp.lo = reinterpret_cast<int32_t*>(ws + w.lo);
+  pp.hi = reinterpret_cast<int32_t*>(ws + w.hi);
+  pp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  pp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  pp.cache_cap = cache_capacity;
+  pp.err = err;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_bshd_map(&tq, pp.q_hat, B, S, Hq, D) || !make_bshd_map(&tk, pp.k_hat, B, S, Hkv, D) ||
+      !make_bshd_map(&tv, v, B, S, Hkv, D))
+    return fail(G3_ERR_CUDA, "prefill: cuTensorMapEncodeTiled unavailable or failed");
+
+  cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill: %s", cudaGetErrorString(e));
+  e = traced("prefill_prologue", st, [&] { return g3::launch_prefill_prologue(pp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill prologue: %s", cudaGetErrorString(e));
+
+  g3::AttnParams ap{};
+  ap.lo = pp.lo;
+  ap.hi = pp.hi;
+  ap.out = static_cast<__nv_bfloat16*>(out);
+  ap.lse = lse;
+  ap.err = err;
+  ap.B = B;
+  ap.S = S;
+  ap.Hq = Hq;
+  ap.Hkv = Hkv;
+  ap.G = G;
+  ap.n_qtiles = (int)n_qtiles;
+  ap.n_groups = G / hpc;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill attention: %s", cudaGetErrorString(e));
+  return G3_OK;
+}
+
+g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new, const float* q_gamma,
+                        const float* k_gamma, void* k_cache, void* v_cache, int32_t cache_capacity,
+                        const int32_t* seq_lens, int32_t max_seq_len, g3_layer_kind layer_kind, int32_t window,
+                        float rope_base, float interp_factor, int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                        void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!q || !k_new || !v_new || !q_gamma || !k_gamma || !k_cache || !v_cache || !seq_lens || !out)
+    return fail(G3_ERR_INVALID_ARG, "decode: a required pointer is NULL");
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || max_seq_len < 1 || cache_capacity < 1)
+    return fail(G3_ERR_INVALID_ARG, "decode: sizes must be positive");
+  if (Hq % Hkv != 0) return fail(G3_ERR_INVALID_ARG, "decode: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
+  if (layer_kind != G3_LAYER_LOCAL && layer_kind != G3_LAYER_GLOBAL)
+    return fail(G3_ERR_INVALID_ARG, "decode: bad layer kind %d", (int)layer_kind);
+  if (layer_kind == G3_LAYER_LOCAL && (window < 1 || cache_capacity != window))
+    return fail(G3_ERR_INVALID_ARG, "decode: local layers need window >= 1 and cache_capacity == window");
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return fail(G3_ERR_INVALID_ARG, "decode: bad rope_base");
+  if (!(interp_factor > 0.f) || !std::isfinite(interp_factor))
+    return fail(G3_ERR_INVALID_ARG, "decode: bad interp_factor");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(G3_ERR_INVALID_ARG, "decode: caches must be 16-byte aligned");
+  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "decode: head_dim %d not built (64, 128)", D);
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4) return fail(G3_ERR_UNSUPPORTED, "decode: group size %d not built (1, 2, 4)", G);
+  if ((size_t)B * Hkv * cache_capacity * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "decode: cache too large");
+
+  DecodeWs w;
+  const int visible_max = layer_kind == G3_LAYER_LOCAL ? std::min(max_seq_len, window) : max_seq_len;
+  decode_ws(B, Hq, Hkv, D, max_seq_len, &w);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(G3_ERR_WORKSPACE, "decode: workspace NULL or not 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(G3_ERR_WORKSPACE, "decode: workspace %zu bytes < required %zu", workspace_bytes, w.total);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  g3::DecodeParams dp{};
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  dp.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  dp.q_gamma = q_gamma;
+  dp.k_gamma = k_gamma;
+  dp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  dp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  dp.cache_cap = cache_capacity;
+  dp.seq_lens = seq_lens;
+  dp.max_seq_len = max_seq_len;
+  dp.kind = (int)layer_kind;
+  dp.window = layer_kind == G3_LAYER_LOCAL ? window : cache_capacity;
+  dp.rope_base = rope_base;
+  dp.interp = interp_factor;
+  dp.B = B;
+  dp.Hq = Hq;
+  dp.Hkv = Hkv;
+  dp.G = G;
+  dp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  dp.n_chunks = w.n_chunks;
+  dp.q_hat = reinterpret_cast<float*>(ws + w.q_hat);
+  dp.n_slots = reinterpret_cast<int32_t*>(ws + w.n_slots);
+  dp.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  dp.part_o = reinterpret_cast<float*>(ws + w.part_o);
+  dp.out = static_cast<__nv_bfloat16*>(out);
+  dp.err = reinterpret_cast<int*>(ws);
+
+  // The split grid only needs to cover the slots a query can see.
+  g3::DecodeParams split = dp;
+  const int split_chunks = (visible_max + g3::kDecodeChunk - 1) / g3::kDecodeChunk;
+
+  cudaError_t e = cudaMemsetAsync(dp.err, 0, 8, st);
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "decode: %s", cudaGetErrorString(e));
+  e = traced("decode_prologue", st, [&] { return g3::launch_decode_prologue(dp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "decode prologue: %s", cudaGetErrorString(e));
+  e = traced("decode_split", st, [&] { return g3::launch_decode_split(split, D, split_chunks, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "decode split: %s", cudaGetErrorString(e));
+  e = traced("decode_combine", st, [&] { return g3::launch_decode_combine(dp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "decode combine: %s", cudaGetErrorString(e));
+  return G3_OK;
+}
+
+g3_status g3attn_check_device_error(void* workspace, void* stream) {
+  if (workspace == nullptr) return fail(G3_ERR_WORKSPACE, "check: workspace is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int h[2] = {0, 0};
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "check: %s", cudaGetErrorString(e));
+  if (h[0] != 0) {
+    const int zero[2] = {0, 0};
+    cudaMemcpy(workspace, zero, sizeof(zero), cudaMemcpyHostToDevice);
+    fail((g3_status)h[0], "device error %d at site %d", h[0], h[1]);
+    return (g3_status)h[0];
+  }
+  return G3_OK;
+}
+
+g3_status g3attn_trace_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  g_trace.enabled = enable != 0;
+  return G3_OK;
+}
+
+int32_t g3attn_trace_collect(g3_kernel_trace* out, int32_t max_entries) {
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  std::vector<g3_kernel_trace> agg;
+  for (TraceEntry& t : g_trace.pending) {
+    float ms = 0.f;
+    cudaEventSynchronize(t.stop);
+    cudaEventElapsedTime(&ms, t.start, t.stop);
+    g3_kernel_trace* slot = nullptr;
+    for (auto& a : agg)
+      if (t.name == a.name) slot = &a;
+    if (slot == nullptr) {
+      agg.push_back(g3_kernel_trace{});
+      slot = &agg.back();
+      std::snprintf(slot->name, sizeof(slot->name), "%s", t.name.c_str());
+    }
+    slot->launches += 1;
+    slot->total_ms += ms;
+    g_trace.pool.push_back(t.start);
+    g_trace.pool.push_back(t.stop);
+  }
+  g_trace.pending.clear();
+  const int n = (int)agg.size() < max_entries ? (int)agg.size() : max_entries;
+  for (int i = 0; i < n && out != nullptr; ++i) out[i] = agg[i];
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// Internal interface between the host API (api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace g3 {
+
+constexpr int kTileRows = 128;       // query rows and key rows per attention tile
+constexpr int kDecodeChunk = 512;    // cached tokens per decode split-KV block
+constexpr size_t kHeaderBytes = 256; // workspace header: error word, site, spare
+
+// Workspace header words (int32): [0] first device error (g3_status),
+// [1] site tag of that error.
+struct PrologueParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* q_gamma;
+  const float* k_gamma;
+  const int32_t* positions;
+  const int32_t* spans;
+  int n_spans;
+  int B, S, Hq, Hkv;
+  int kind;            // 0 local, 1 global
+  int window;
+  double rope_base;
+  double interp;
+  __nv_bfloat16* q_hat;  // [B,S,Hq,D]
+  __nv_bfloat16* k_hat;  // [B,S,Hkv,D]
+  int32_t* lo;           // [B,S] first visible key of each row
+  int32_t* hi;           // [B,S] last visible key of each row
+  __nv_bfloat16* k_cache;
+  __nv_bfloat16* v_cache;
+  int cache_cap;
+  int* err;
+};
+
+struct AttnParams {
+  const int32_t* lo;
+  const int32_t* hi;
+  __nv_bfloat16* out;  // [B,S,Hq,D]
+  float* lse;          // [B,Hq,S] or null
+  int* err;
+  int B, S, Hq, Hkv, G;
+  int n_qtiles;
+  int n_groups;        // G / heads_per_cta
+  float scale_log2;    // log2(e) / sqrt(D)
+};
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  const float* q_gamma;
+  const float* k_gamma;
+  __nv_bfloat16* k_cache;  // [B,Hkv,cap,D]
+  __nv_bfloat16* v_cache;
+  int cache_cap;
+  const int32_t* seq_lens;
+  int max_seq_len;
+  int kind;
+  int window;
+  double rope_base;
+  double interp;
+  int B, Hq, Hkv, G;
+  float scale_log2;
+  int n_chunks;            // ceil(max visible slots / kDecodeChunk)
+  float* q_hat;            // [B,Hq,D] fp32, pre-multiplied by scale_log2
+  int32_t* n_slots;        // [B] visible cache slots (0 = invalid sequence)
+  float* part_ml;          // [B,Hq,n_chunks,2]  (max, sum) in log2 units
+  float* part_o;           // [B,Hq,n_chunks,D]
+  __nv_bfloat16* out;      // [B,Hq,D]
+  int* err;
+};
+
+// Launchers return the launch status; `name` receives a static kernel name
+// for tracing.
+cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st);
+cudaError_t launch_prefill_attention(const AttnParams& p, int D, int heads_per_cta, const CUtensorMap& tm_q,
+                                     const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
+size_t prefill_attention_smem_bytes(int D, int heads_per_cta);
+
+cudaError_t launch_decode_prologue(const DecodeParams& p, int D, cudaStream_t st);
+cudaError_t launch_decode_split(const DecodeParams& p, int D, int grid_chunks, cudaStream_t st);
+cudaError_t launch_decode_combine(const DecodeParams& p, int D, cudaStream_t st);
+
+}  // namespace g3

@@ -1,0 +1,175 @@
+/*
+ * g3attn -- attention of Gemma 3's 5:1 local/global decoder block on B200.
+ *
+ * One call computes one attention layer of the block:
+ *   1. QK-norm: per token and head, q and k are divided by their RMS over
+ *      head_dim (eps 1e-6) and multiplied by a per-feature gain (Gemma 3
+ *      Technical Report, section 2 "Model Architecture"; eps and dim from the
+ *      q_norm/k_norm lines of the printouts on "Gemma explained: what's new in
+ *      Gemma 3").
+ *   2. RoPE with the layer's own base and linear position interpolation:
+ *      pairs (d, d + D/2) rotate by (p / interp) * base^(-2d/D) (Technical
+ *      Report, section 2 "Long context": local base 10k, global base 1M,
+ *      interpolation for the global layers).
+ *   3. Masked softmax attention with scale 1/sqrt(D).  Key j is visible from
+ *      query i iff (j <= i and (GLOBAL or i - j < window)) or i and j lie in
+ *      the same image span (Technical Report, sections 1 and 2 "5:1
+ *      interleaving"; "Gemma explained", section "Vision encoder and
+ *      processing": bidirectional attention over image tokens).
+ *   4. Grouped-query attention: query head h reads key/value head h / G,
+ *      G = Hq / Hkv.
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *     owned by the caller.  bf16 tensors are raw IEEE bfloat16 (uint16).
+ *     q, k, v, out, k_cache, v_cache must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous: G3_OK means the work was enqueued.
+ *   - The library allocates no device memory and keeps no per-call state.
+ *     Scratch lives in the caller's `workspace`, sized by the matching
+ *     *_workspace_size() query; one workspace must not be shared by two
+ *     calls that may run concurrently.
+ *   - Argument errors are detected on the host before any launch and return
+ *     G3_ERR_INVALID_ARG or G3_ERR_UNSUPPORTED; nothing is enqueued then.
+ *     Errors that depend on device-resident values (image spans that are
+ *     unsorted, overlapping or out of range; sequence lengths out of range)
+ *     and bounded-wait timeouts inside the kernels are recorded in the
+ *     workspace and reported by g3attn_check_device_error().  A kernel that
+ *     meets such an error writes no output for the affected rows but never
+ *     reads or writes out of bounds.
+ *   - Launch failures return G3_ERR_CUDA; g3attn_last_error() gives detail.
+ */
+#ifndef G3ATTN_H
+#define G3ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  G3_OK = 0,
+  G3_ERR_INVALID_ARG = 1,  /* bad pointer, size, shape, or device-side value */
+  G3_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim or group size    */
+  G3_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small     */
+  G3_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed           */
+  G3_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel gave up         */
+} g3_status;
+
+typedef enum { G3_LAYER_LOCAL = 0, G3_LAYER_GLOBAL = 1 } g3_layer_kind;
+
+/* ------------------------------------------------------------------ prefill
+ * Bytes of workspace g3attn_prefill needs for these sizes (0 if the sizes are
+ * invalid).  The workspace must be 256-byte aligned.
+ */
+size_t g3attn_prefill_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D);
+
+/*
+ * Prefill: attention of all S query tokens of B sequences for one layer.
+ *
+ *   q          bf16 [B, S, Hq,  D]  raw query projections (before norm/RoPE)
+ *   k, v       bf16 [B, S, Hkv, D]  raw key projections, value projections
+ *   q_gamma    fp32 [D]             query norm gain (multiplier)
+ *   k_gamma    fp32 [D]             key norm gain
+ *   positions  int32 [B, S]         RoPE positions (the mask uses token index)
+ *   layer_kind G3_LAYER_LOCAL (sliding window) or G3_LAYER_GLOBAL (causal)
+ *   window     keys visible to a local query, itself included (>= 1); ignored
+ *              for GLOBAL layers
+ *   rope_base  > 0;  interp_factor > 0 (positions are divided by it)
+ *   image_spans int32 [B, n_spans, 2] half-open [start, end) per sequence,
+ *              sorted, disjoint, 0 <= start < end <= S; NULL iff n_spans == 0
+ *   B, S, Hq, Hkv, D   S >= 1, Hq % Hkv == 0, D in {64, 128}
+ *   out        bf16 [B, S, Hq, D]
+ *   lse        optional fp32 [B, Hq, S]: natural-log sum of exp of the scaled
+ *              scores of each row (NULL to skip)
+ *   k_cache, v_cache optional bf16 [B, Hkv, cache_capacity, D]: when given,
+ *              the rotated keys and the values are also written there, for a
+ *              later g3attn_decode.  GLOBAL: token t goes to slot t and
+ *              cache_capacity >= S.  LOCAL: a ring of cache_capacity == window
+ *              slots; token t goes to slot t % window and only the last
+ *              min(S, window) tokens are written.  Both NULL to skip.
+ *   workspace  >= g3attn_prefill_workspace_size(B, S, Hq, Hkv, D) bytes
+ */
+g3_status g3attn_prefill(const void* q, const void* k, const void* v,
+                         const float* q_gamma, const float* k_gamma,
+                         const int32_t* positions,
+                         g3_layer_kind layer_kind, int32_t window,
+                         float rope_base, float interp_factor,
+                         const int32_t* image_spans, int32_t n_spans,
+                         int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                         void* out, float* lse,
+                         void* k_cache, void* v_cache, int32_t cache_capacity,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------- decode
+ * Bytes of workspace g3attn_decode needs (0 if the sizes are invalid).
+ */
+size_t g3attn_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                                    int32_t max_seq_len);
+
+/*
+ * Decode: one new token per sequence, attending to its cached context.
+ *
+ *   q          bf16 [B, Hq, D]   raw query of the new token
+ *   k_new, v_new bf16 [B, Hkv, D] raw key / value of the new token
+ *   q_gamma, k_gamma fp32 [D]
+ *   k_cache, v_cache bf16 [B, Hkv, cache_capacity, D]: rotated keys and values
+ *              of earlier tokens.  GLOBAL: token t in slot t.  LOCAL: ring of
+ *              cache_capacity == window slots, token t in slot t % window.
+ *              The call first writes the new token's rotated key and its value
+ *              into slot L-1 (GLOBAL) or (L-1) % window (LOCAL), then attends.
+ *   seq_lens   int32 [B] on the device: tokens of each sequence including the
+ *              new one (its position and index are L-1); 1 <= L <= max_seq_len,
+ *              and L <= cache_capacity for GLOBAL layers
+ *   max_seq_len host-side upper bound of seq_lens, used to size the launch
+ *   out        bf16 [B, Hq, D]
+ *   workspace  >= g3attn_decode_workspace_size(B, Hq, Hkv, D, max_seq_len)
+ * A sequence whose length is out of range gets a zero output row, its cache is
+ * left untouched, and G3_ERR_INVALID_ARG is recorded for
+ * g3attn_check_device_error().
+ */
+g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new,
+                        const float* q_gamma, const float* k_gamma,
+                        void* k_cache, void* v_cache, int32_t cache_capacity,
+                        const int32_t* seq_lens, int32_t max_seq_len,
+                        g3_layer_kind layer_kind, int32_t window,
+                        float rope_base, float interp_factor,
+                        int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                        void* out,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------- checking
+ * Synchronises `stream`, then returns (and clears) the first device-side error
+ * recorded in `workspace` by the last prefill/decode call that used it:
+ * G3_OK, G3_ERR_INVALID_ARG (bad spans or sequence lengths) or G3_ERR_TIMEOUT.
+ */
+g3_status g3attn_check_device_error(void* workspace, void* stream);
+
+/* Static text for a status code. */
+const char* g3attn_status_string(g3_status status);
+
+/* Detail of the last host-side error on the calling thread ("" if none). */
+const char* g3attn_last_error(void);
+
+/* ------------------------------------------------------------------ tracing
+ * When enabled, every kernel the library launches is bracketed by a pair of
+ * CUDA events on its own stream; g3attn_trace_collect() synchronises those
+ * events and returns, per kernel name, the number of launches and their summed
+ * device time since the last collect (which also resets the counts).
+ */
+typedef struct {
+  char name[48];
+  int64_t launches;
+  double total_ms;
+} g3_kernel_trace;
+
+g3_status g3attn_trace_enable(int enable);
+int32_t g3attn_trace_collect(g3_kernel_trace* out, int32_t max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* G3ATTN_H */

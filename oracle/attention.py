@@ -181,19 +181,26 @@ def prefill_rows(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_base, 
     if None), the same for every sequence.
     Returns (out [B, R, Hq, D], lse [B, Hq, R]) in float64.
     """
-    qh, kh, vf = _prepare(q, k, v, q_gamma, k_gamma, positions, rope_base, interp)
-    B, S, Hq, D = qh.shape
+    B, S, Hq, D = q.shape
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
     out = np.empty((B, rows.size, Hq, D))
     lse = np.empty((B, Hq, rows.size))
     sp = None if spans is None else _i64(spans)
+    pos = _f64(positions)
     for b in range(B):
+        # Steps 1-2 for the keys of this sequence and for the requested query
+        # rows only (a query row's result needs no other query row).
+        kh = rope(qk_rmsnorm(k[b], k_gamma), pos[b], rope_base, interp)
+        qsel = rope(qk_rmsnorm(q[b][rows], q_gamma), pos[b][rows], rope_base, interp)
+        qh = np.zeros((S, Hq, D))
+        qh[rows] = qsel
         sid = span_ids(S, None if sp is None else sp[b])
-        kh_hm = np.ascontiguousarray(kh[b].transpose(1, 0, 2))
-        v_hm = np.ascontiguousarray(vf[b].transpose(1, 0, 2))
+        kh_hm = np.ascontiguousarray(kh.transpose(1, 0, 2))
+        v_hm = np.ascontiguousarray(_f64(v[b]).transpose(1, 0, 2))
+        del kh
         for g0 in range(0, rows.size, row_group):
             sel = rows[g0:g0 + row_group]
-            o, ls = _attend_rows(qh[b], kh_hm, v_hm, sel, kind, window, sid, S)
+            o, ls = _attend_rows(qh, kh_hm, v_hm, sel, kind, window, sid, S)
             out[b, g0:g0 + sel.size] = o
             lse[b, :, g0:g0 + sel.size] = ls
     return out, lse
