@@ -118,6 +118,22 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
+# ------------------------------------------------------- multi-rank helpers
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (the slowest rank's time)."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist = torch.distributed
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Units per second of the whole job: every rank does the same work."""
+    return units_per_rank_step * steps * world / (ms_max * 1e-3)
+
+
 # ------------------------------------------------------------ CPU baselines
 def blas_threads() -> int:
     try:
@@ -218,11 +234,8 @@ def run_gpu(args, rank, world, local_rank):
     trace = g3.trace_collect()
     if g3.check_device_error(ws) != 0:
         raise RuntimeError("device error in the timed region")
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = block_flops * args.steps * world / (ms_max * 1e-3) / 1e12
+    ms_max = max_over_ranks(ms, dev)
+    value = weak_scaling_rate(block_flops, args.steps, world, ms_max) / 1e12
 
     n_attn, attn_ms = trace.get("prefill_attention", (0, 0.0))
     achieved = block_flops * args.steps / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
@@ -269,10 +282,8 @@ def run_gpu(args, rank, world, local_rank):
     e1.record(stream)
     barrier()
     wall = time.perf_counter() - w0
-    e2e_ms = torch.tensor([max(e0.elapsed_time(e1), wall * 1e3)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = block_flops * e2e_steps * world / (float(e2e_ms.item()) * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(max(e0.elapsed_time(e1), wall * 1e3), dev)
+    e2e_value = weak_scaling_rate(block_flops, e2e_steps, world, e2e_ms) / 1e12
     del host
 
     # ---- decode block step on the 64 x (4K..128K) workload
@@ -350,11 +361,8 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
     if world > 1:
         torch.distributed.barrier()
     trace = g3.trace_collect()
-    ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
-    ms = float(ms.item())
-    gbs = step_bytes * args.steps * world / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    gbs = weak_scaling_rate(step_bytes, args.steps, world, ms) / 1e9
     n_split, split_ms = trace.get("decode_split", (0, 0.0))
     ach = step_bytes * args.steps / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
     del caches
