@@ -45,6 +45,8 @@ _SIGS = {
     "g3attn_decode_workspace_size": (_sz, [_i32] * 5),
     "g3attn_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, ctypes.c_int, _i32,
                                      _f32, _f32, _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
+    "g3attn_decode_no_alloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, ctypes.c_int,
+                                              _i32, _f32, _f32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "g3attn_check_device_error": (ctypes.c_int, [_vp, _vp]),
     "g3attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "g3attn_last_error": (ctypes.c_char_p, []),

@@ -146,6 +146,8 @@ bool supported_d(int D) { return D == 64 || D == 128; }
 
 }  // namespace
 
+void g3::set_last_error(const char* msg) { g_last_error = msg; }
+
 extern "C" {
 
 const char* g3attn_status_string(g3_status s) {

@@ -84,6 +84,9 @@ cudaError_t launch_prefill_attention(const AttnParams& p, int D, int heads_per_c
                                      const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
 size_t prefill_attention_smem_bytes(int D, int heads_per_cta);
 
+// Sets the calling thread's g3attn_last_error() text.
+void set_last_error(const char* msg);
+
 cudaError_t launch_decode_prologue(const DecodeParams& p, int D, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeParams& p, int D, int grid_chunks, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeParams& p, int D, cudaStream_t st);

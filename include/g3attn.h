@@ -140,6 +140,34 @@ g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new,
                         void* out,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Decode without a caller workspace.  (The sources describe the model only;
+ * this entry point has no counterpart there and exists for callers that
+ * cannot allocate device memory: a plugin whose host framework owns all device
+ * memory through its own pool, a serving loop that may not call cudaMalloc
+ * because it can synchronise the device, a C caller with no allocator.)
+ *
+ * Same arguments and results as g3attn_decode, minus the workspace: the
+ * scratch lives in a 16 MiB device array inside the library, which every GPU
+ * that loads the library keeps until the process exits.  The call allocates
+ * nothing.  Sizes whose scratch (g3attn_decode_workspace_size) exceeds
+ * 16 MiB return G3_ERR_UNSUPPORTED with a message in g3attn_last_error().
+ * All calls on a device share the array and it keeps the last call's
+ * contents, so calls that may overlap on the GPU race and must be ordered by
+ * the caller.  The first call on each device looks up the array's address;
+ * make it before any stream capture starts.  Out-of-range sequence lengths
+ * give zero output rows (their device-side status is not reported by this
+ * variant).
+ */
+g3_status g3attn_decode_no_alloc(const void* q, const void* k_new, const void* v_new,
+                                 const float* q_gamma, const float* k_gamma,
+                                 void* k_cache, void* v_cache, int32_t cache_capacity,
+                                 const int32_t* seq_lens, int32_t max_seq_len,
+                                 g3_layer_kind layer_kind, int32_t window,
+                                 float rope_base, float interp_factor,
+                                 int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                                 void* out, void* stream);
+
 /* ----------------------------------------------------------------- checking
  * Synchronises `stream`, then returns (and clears) the first device-side error
  * recorded in `workspace` by the last prefill/decode call that used it:
