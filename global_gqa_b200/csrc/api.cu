@@ -104,7 +104,7 @@ bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int 
 
 // ---------------------------------------------------------- workspace maps
 struct PrefillWs {
-  size_t lo, hi, q_hat, k_hat, total;
+  size_t lo, hi, table, q_hat, k_hat, total;
 };
 bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w) {
   if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || D < 1) return false;
@@ -114,6 +114,8 @@ bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w) {
   off = align_up(off + rows * 4, 1024);
   w->hi = off;
   off = align_up(off + rows * 4, 1024);
+  w->table = off;
+  off = align_up(off + rows * (D / 2) * 8, 1024);
   w->q_hat = off;
   off = align_up(off + rows * Hq * D * 2, 1024);
   w->k_hat = off;
@@ -242,10 +244,12 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   pp.window = layer_kind == G3_LAYER_LOCAL ? window : S;
   pp.rope_base = rope_base;
   pp.interp = interp_factor;
+  for (int f = 0; f < D / 2; ++f) pp.inv_freq[f] = std::pow((double)rope_base, -2.0 * f / D);
   pp.q_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.q_hat);
   pp.k_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.k_hat);
   pp.lo = reinterpret_cast<int32_t*>(ws + w.lo);
   pp.hi = reinterpret_cast<int32_t*>(ws + w.hi);
+  pp.rope_table = reinterpret_cast<float2*>(ws + w.table);
   pp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
   pp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
   pp.cache_cap = cache_capacity;

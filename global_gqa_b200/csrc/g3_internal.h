@@ -29,10 +29,12 @@ struct PrologueParams {
   int window;
   double rope_base;
   double interp;
+  double inv_freq[64];   // base^(-2f/D), f < D/2, computed on the host in double
   __nv_bfloat16* q_hat;  // [B,S,Hq,D]
   __nv_bfloat16* k_hat;  // [B,S,Hkv,D]
   int32_t* lo;           // [B,S] first visible key of each row
   int32_t* hi;           // [B,S] last visible key of each row
+  float2* rope_table;    // [B,S,D/2] (cos, sin) of each rotation angle
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   int cache_cap;

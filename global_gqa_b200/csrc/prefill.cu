@@ -1,7 +1,6 @@
-// Prefill path of the Gemma 3 block attention on sm_100a.
+// Prefill attention of the Gemma 3 block on sm_100a (the prologue that
+// normalises and rotates q and k is in prologue.cu).
 //
-//   prefill_prologue : QK-RMSNorm + RoPE of q and k (bf16 out), per-row visible
-//                      key interval [lo, hi], optional KV-cache fill.
 //   prefill_attention: warp-specialised flash attention.  TMA (no multicast)
 //                      streams 128-row K/V tiles, one thread issues tcgen05.mma
 //                      for S = Q K^T and O += P V with accumulators in tensor
@@ -27,145 +26,6 @@
 #include "sm100_ptx.cuh"
 
 namespace g3 {
-
-// ========================================================== prologue kernel
-constexpr int kPrologueTokens = 4;     // tokens per block
-constexpr int kPrologueThreads = 256;  // 8 warps
-
-template <int D>
-__global__ void __launch_bounds__(kPrologueThreads) prefill_prologue_kernel(PrologueParams p) {
-  constexpr int H2 = D / 2;
-  constexpr int PER = D / 64;  // elements per lane in each half of the head
-  __shared__ float s_cos[kPrologueTokens][H2];
-  __shared__ float s_sin[kPrologueTokens][H2];
-
-  const int b = blockIdx.y;
-  const int t0 = blockIdx.x * kPrologueTokens;
-  const int tid = threadIdx.x;
-
-  // Rotation angles in double: theta = (p / interp) * base^(-2f/D), then sin
-  // and cos in double and rounded to fp32.
-  for (int idx = tid; idx < kPrologueTokens * H2; idx += blockDim.x) {
-    const int tt = idx / H2, f = idx % H2, t = t0 + tt;
-    float c = 1.f, s = 0.f;
-    if (t < p.S) {
-      const double inv_freq = exp(-2.0 * f / D * log(p.rope_base));
-      const double theta = (double)p.positions[(size_t)b * p.S + t] / p.interp * inv_freq;
-      double sd, cd;
-      sincos(theta, &sd, &cd);
-      c = (float)cd;
-      s = (float)sd;
-    }
-    s_cos[tt][f] = c;
-    s_sin[tt][f] = s;
-  }
-
-  // Visible interval of each row of this block.
-  if (tid < kPrologueTokens) {
-    const int t = t0 + tid;
-    if (t < p.S) {
-      int lo = (p.kind == 1) ? 0 : max(0, t - p.window + 1);
-      int hi = t;
-      const int32_t* sp = p.spans + (size_t)b * p.n_spans * 2;
-      for (int k = 0; k < p.n_spans; ++k) {
-        const int st = sp[2 * k], en = sp[2 * k + 1];
-        if (st <= t && t < en) {
-          lo = min(lo, max(st, 0));
-          hi = max(hi, min(en, p.S) - 1);
-          break;
-        }
-      }
-      p.lo[(size_t)b * p.S + t] = lo;
-      p.hi[(size_t)b * p.S + t] = hi;
-    }
-  }
-  // Span validation for this sequence (one thread of its first block).
-  if (blockIdx.x == 0 && tid == 32 && p.n_spans > 0) {
-    const int32_t* sp = p.spans + (size_t)b * p.n_spans * 2;
-    int prev_end = 0;
-    bool ok = true;
-    for (int k = 0; k < p.n_spans; ++k) {
-      const int st = sp[2 * k], en = sp[2 * k + 1];
-      ok = ok && st >= prev_end && st < en && en <= p.S;
-      prev_end = en;
-    }
-    if (!ok) record_error(p.err, kErrInvalid, 100);
-  }
-  __syncthreads();
-
-  const int warp = tid >> 5, lane = tid & 31;
-  const int heads = p.Hq + p.Hkv;
-  for (int r = warp; r < kPrologueTokens * heads; r += kPrologueThreads / 32) {
-    const int tt = r / heads, h = r % heads, t = t0 + tt;
-    if (t >= p.S) continue;
-    const bool is_q = h < p.Hq;
-    const int hh = is_q ? h : h - p.Hq;
-    const int H = is_q ? p.Hq : p.Hkv;
-    const size_t row = ((size_t)b * p.S + t) * H + hh;
-    const __nv_bfloat16* src = (is_q ? p.q : p.k) + row * D;
-    const float* gam = is_q ? p.q_gamma : p.k_gamma;
-    float x1[PER], x2[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      x1[e] = __bfloat162float(src[lane * PER + e]);
-      x2[e] = __bfloat162float(src[H2 + lane * PER + e]);
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) ss += x1[e] * x1[e] + x2[e] * x2[e];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float rinv = rsqrtf(ss / (float)D + 1e-6f);
-    __nv_bfloat16* dst = (is_q ? p.q_hat : p.k_hat) + row * D;
-    __nv_bfloat16 o1[PER], o2[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      const int d = lane * PER + e;
-      const float y1 = x1[e] * rinv * gam[d];
-      const float y2 = x2[e] * rinv * gam[d + H2];
-      const float c = s_cos[tt][d], s = s_sin[tt][d];
-      o1[e] = __float2bfloat16_rn(y1 * c - y2 * s);
-      o2[e] = __float2bfloat16_rn(y1 * s + y2 * c);
-      dst[d] = o1[e];
-      dst[d + H2] = o2[e];
-    }
-    if (!is_q && p.k_cache != nullptr) {
-      bool write;
-      int slot;
-      if (p.kind == 1) {
-        write = t < p.cache_cap;
-        slot = t;
-      } else {
-        write = t >= p.S - p.cache_cap;
-        slot = t % p.cache_cap;
-      }
-      if (write) {
-        const size_t crow = ((size_t)b * p.Hkv + hh) * p.cache_cap + slot;
-        const __nv_bfloat16* vsrc = p.v + row * D;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) {
-          const int d = lane * PER + e;
-          p.k_cache[crow * D + d] = o1[e];
-          p.k_cache[crow * D + d + H2] = o2[e];
-          p.v_cache[crow * D + d] = vsrc[d];
-          p.v_cache[crow * D + d + H2] = vsrc[d + H2];
-        }
-      }
-    }
-  }
-}
-
-cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st) {
-  dim3 grid((p.S + kPrologueTokens - 1) / kPrologueTokens, p.B);
-  if (D == 128) {
-    prefill_prologue_kernel<128><<<grid, kPrologueThreads, 0, st>>>(p);
-  } else if (D == 64) {
-    prefill_prologue_kernel<64><<<grid, kPrologueThreads, 0, st>>>(p);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
 
 // ========================================================= attention kernel
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
@@ -254,7 +114,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
+  // Producer / MMA warpgroup gives registers to the two softmax warpgroups
+  // (128 x 56 + 256 x 224 = 384 x 168, the launch's register budget).  Each
+  // role runs inside the branch that set its register count.
+  if (warp < 4) {
+    setmaxnreg_dec<56>();
+   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
@@ -356,7 +221,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(&bars->drain, 0, &no_abort, p.err, 16);
     }
-  } else if (warp >= 4 && warp < 4 + 4 * HPC) {
+   }
+  } else {
+    setmaxnreg_inc<224>();
+   if (warp < 4 + 4 * HPC) {
     // ------------------------------------------------------------- softmax
     const int h = (warp - 4) >> 2;
     const int lane_base = (warp & 3) * 32;
@@ -389,9 +257,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (j < lo_i || j > hi_i) sv[c] = -INFINITY;
         }
       }
-      float mx = sv[0];
+      float mx0 = fmax3(sv[0], sv[1], sv[2]), mx1 = fmax3(sv[3], sv[4], sv[5]);
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+      for (int c = 6; c < 126; c += 4) {
+        mx0 = fmax3(mx0, sv[c], sv[c + 1]);
+        mx1 = fmax3(mx1, sv[c + 2], sv[c + 3]);
+      }
+      const float mx = fmax3(fmax3(mx0, mx1, sv[126]), sv[127], sv[127]);
       const float m_new = fmaxf(m_ref, mx * sc);
       const bool first = (m_ref == -INFINITY);
       const bool need = !first && (m_new > m_ref + 8.f);
@@ -414,16 +286,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float sum = 0.f;
+      // Exponentials two at a time (one f16x2 exp-unit operation per pair),
+      // scaling and sums as packed fp32x2 operations, two partial sum pairs.
+      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
       uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(sv[2 * c], sc, -m_use));
-        const float p1 = ex2_approx(fmaf(sv[2 * c + 1], sc, -m_use));
-        sum += p0 + p1;
+        float x0, x1, p0, p1;
+        ffma2_bcast(sv[2 * c], sv[2 * c + 1], sc, -m_use, x0, x1);
+        ex2_pair_f16(x0, x1, p0, p1);
+        if (c & 1) {
+          fadd2(sb0, sb1, p0, p1);
+        } else {
+          fadd2(sa0, sa1, p0, p1);
+        }
         pk[c] = pack_bf16x2(p0, p1);
       }
-      l_sum += sum;
+      l_sum += (sa0 + sa1) + (sb0 + sb1);
       tmem_st32(t_lane + s_col, pk);
       tmem_st32(t_lane + s_col + 32, pk + 32);
       tmem_wait_st();
@@ -452,11 +331,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (valid && p.lse != nullptr)
         p.lse[((size_t)b * p.Hq + hq) * p.S + row] = (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
     }
+   }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

@@ -1,0 +1,203 @@
+// Prefill prologue: QK-RMSNorm + RoPE of q and k, the per-row visible key
+// interval, and the optional KV-cache fill, in two launches:
+//
+//   rope_table  : per token, (cos, sin) of every rotation angle, formed and
+//                 evaluated in double and stored as fp32 [B, S, D/2] (a few MB,
+//                 read back from L2); the token's visible interval; validation
+//                 of the image spans.
+//   qk_norm_rope: bandwidth-bound pass over every (token, head) row of q and k.
+//                 One warp per token: the token's cos/sin are loaded once into
+//                 registers and serve all of its Hq + Hkv rows; eight row steps
+//                 of 8-byte loads per lane are in flight; no block-wide sync.
+//
+// Norm (Gemma 3 Technical Report, section 2; eps and dim from the q_norm /
+// k_norm lines of "Gemma explained: what's new in Gemma 3"): x / sqrt(mean(x^2)
+// + 1e-6) * gamma in fp32.  RoPE (Technical Report, section 2 "Long
+// context"): pair (d, d + D/2) turns by theta = (p / interp) * base^(-2d/D);
+// the rotation is done in fp32 and the result rounded to bf16.
+//
+// Visible interval of row i: the causal window [max(0, i-W+1), i] ([0, i] on a
+// global layer) joined with the row's image span, which is contiguous because
+// both contain i (Technical Report sections 1 and 2; "Gemma explained",
+// section "Vision encoder and processing").
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "g3_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace g3 {
+
+constexpr int kTableThreads = 256;
+constexpr int kRowThreads = 256;  // 8 warps, one token each at a time
+constexpr int kRowUnroll = 8;     // row steps in flight per warp
+
+template <int D>
+__global__ void __launch_bounds__(kTableThreads) rope_table_kernel(PrologueParams p) {
+  constexpr int H2 = D / 2;
+  const size_t idx = (size_t)blockIdx.x * kTableThreads + threadIdx.x;
+  const size_t total = (size_t)p.B * p.S * H2;
+  if (idx >= total) return;
+  const size_t bt = idx / H2;
+  const int f = (int)(idx % H2);
+  const int b = (int)(bt / p.S), t = (int)(bt % p.S);
+  const double theta = (double)p.positions[bt] / p.interp * p.inv_freq[f];
+  double sd, cd;
+  sincos(theta, &sd, &cd);
+  p.rope_table[idx] = make_float2((float)cd, (float)sd);
+
+  if (f == 0) {
+    int lo = (p.kind == 1) ? 0 : max(0, t - p.window + 1);
+    int hi = t;
+    const int32_t* sp = p.spans + (size_t)b * p.n_spans * 2;
+    for (int k = 0; k < p.n_spans; ++k) {
+      const int st = sp[2 * k], en = sp[2 * k + 1];
+      if (st <= t && t < en) {
+        lo = min(lo, max(st, 0));
+        hi = max(hi, min(en, p.S) - 1);
+        break;
+      }
+    }
+    p.lo[bt] = lo;
+    p.hi[bt] = hi;
+    if (t == 0 && p.n_spans > 0) {
+      int prev_end = 0;
+      bool ok = true;
+      for (int k = 0; k < p.n_spans; ++k) {
+        const int st = sp[2 * k], en = sp[2 * k + 1];
+        ok = ok && st >= prev_end && st < en && en <= p.S;
+        prev_end = en;
+      }
+      if (!ok) record_error(p.err, kErrInvalid, 100);
+    }
+  }
+}
+
+__device__ __forceinline__ void unpack4_bf16(const uint2 u, float* f) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+
+__device__ __forceinline__ uint2 pack4_bf16(const float* f) {
+  return make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kRowThreads, 3) qk_norm_rope_kernel(PrologueParams p) {
+  constexpr int H2 = D / 2;
+  constexpr int LPR = D / 8;     // lanes per row: each holds 4 features of each half
+  constexpr int RPW = 32 / LPR;  // rows per warp step
+  const int lane = threadIdx.x & 31;
+  const int li = lane % LPR, sub = lane / LPR;
+  const int d1 = li * 4;  // this lane: features d1..d1+3 and H2+d1..H2+d1+3
+  const int heads = p.Hq + p.Hkv;
+  const int n_tokens = p.B * p.S;
+  const int warps_total = gridDim.x * (kRowThreads / 32);
+
+  for (int bt = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); bt < n_tokens; bt += warps_total) {
+    const float4* tab = reinterpret_cast<const float4*>(p.rope_table + (size_t)bt * H2 + d1);
+    const float4 cs0 = __ldg(tab), cs1 = __ldg(tab + 1);
+    const float c[4] = {cs0.x, cs0.z, cs1.x, cs1.z};
+    const float s[4] = {cs0.y, cs0.w, cs1.y, cs1.w};
+    const __nv_bfloat16* qrow = p.q + (size_t)bt * p.Hq * D;
+    const __nv_bfloat16* krow = p.k + (size_t)bt * p.Hkv * D;
+
+    for (int h0 = 0; h0 < heads; h0 += RPW * kRowUnroll) {
+      uint2 xa[kRowUnroll], xb[kRowUnroll];
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        const int h = h0 + u * RPW + sub;
+        if (h < heads) {
+          const __nv_bfloat16* src = h < p.Hq ? qrow + h * D : krow + (h - p.Hq) * D;
+          xa[u] = __ldg(reinterpret_cast<const uint2*>(src + d1));
+          xb[u] = __ldg(reinterpret_cast<const uint2*>(src + H2 + d1));
+        } else {
+          xa[u] = xb[u] = make_uint2(0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        float x[8];
+        unpack4_bf16(xa[u], x);
+        unpack4_bf16(xb[u], x + 4);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const int h = h0 + u * RPW + sub;
+        if (h >= heads) continue;
+        const bool is_q = h < p.Hq;
+        const float rinv = rsqrtf(ss * (1.0f / D) + 1e-6f);
+        const float* gam = is_q ? p.q_gamma : p.k_gamma;
+        const float4 ga = __ldg(reinterpret_cast<const float4*>(gam + d1));
+        const float4 gb = __ldg(reinterpret_cast<const float4*>(gam + H2 + d1));
+        const float g1[4] = {ga.x, ga.y, ga.z, ga.w};
+        const float g2[4] = {gb.x, gb.y, gb.z, gb.w};
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float y1 = x[e] * rinv * g1[e];
+          const float y2 = x[4 + e] * rinv * g2[e];
+          o[e] = y1 * c[e] - y2 * s[e];
+          o[4 + e] = y1 * s[e] + y2 * c[e];
+        }
+        const uint2 lo4 = pack4_bf16(o), hi4 = pack4_bf16(o + 4);
+        if (is_q) {
+          __nv_bfloat16* dst = p.q_hat + ((size_t)bt * p.Hq + h) * D;
+          *reinterpret_cast<uint2*>(dst + d1) = lo4;
+          *reinterpret_cast<uint2*>(dst + H2 + d1) = hi4;
+        } else {
+          const int kh = h - p.Hq;
+          const size_t row = (size_t)bt * p.Hkv + kh;
+          __nv_bfloat16* dst = p.k_hat + row * D;
+          *reinterpret_cast<uint2*>(dst + d1) = lo4;
+          *reinterpret_cast<uint2*>(dst + H2 + d1) = hi4;
+          if (p.k_cache != nullptr) {
+            const int b = bt / p.S, t = bt % p.S;
+            const bool write = (p.kind == 1) ? (t < p.cache_cap) : (t >= p.S - p.cache_cap);
+            if (write) {
+              const int slot = (p.kind == 1) ? t : t % p.cache_cap;
+              const size_t crow = ((size_t)b * p.Hkv + kh) * p.cache_cap + slot;
+              *reinterpret_cast<uint2*>(p.k_cache + crow * D + d1) = lo4;
+              *reinterpret_cast<uint2*>(p.k_cache + crow * D + H2 + d1) = hi4;
+              const __nv_bfloat16* vsrc = p.v + row * D;
+              *reinterpret_cast<uint2*>(p.v_cache + crow * D + d1) =
+                  __ldg(reinterpret_cast<const uint2*>(vsrc + d1));
+              *reinterpret_cast<uint2*>(p.v_cache + crow * D + H2 + d1) =
+                  __ldg(reinterpret_cast<const uint2*>(vsrc + H2 + d1));
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st) {
+  const size_t table_threads = (size_t)p.B * p.S * (D / 2);
+  const unsigned table_blocks = (unsigned)((table_threads + kTableThreads - 1) / kTableThreads);
+  const long long tokens = (long long)p.B * p.S;
+  long long blocks = (tokens + (kRowThreads / 32) - 1) / (kRowThreads / 32);
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (D == 128) {
+    rope_table_kernel<128><<<table_blocks, kTableThreads, 0, st>>>(p);
+    qk_norm_rope_kernel<128><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
+  } else if (D == 64) {
+    rope_table_kernel<64><<<table_blocks, kTableThreads, 0, st>>>(p);
+    qk_norm_rope_kernel<64><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace g3
