@@ -4,8 +4,8 @@
 //   prefill_attention: warp-specialised flash attention.  TMA (no multicast)
 //                      streams 128-row K/V tiles, one thread issues tcgen05.mma
 //                      for S = Q K^T and O += P V with accumulators in tensor
-//                      memory, and one warpgroup per query head of the GQA group
-//                      runs the fp32 online softmax.  The KV tiles a query tile
+//                      memory, and eight warps per query head of the GQA pair
+//                      run the fp32 online softmax (four threads per row).  The KV tiles a query tile
 //                      visits are exactly those its rows' visible intervals
 //                      touch; tiles fully inside every row's interval skip the
 //                      per-element mask.
@@ -24,14 +24,16 @@
 
 #include "g3_internal.h"
 #include "sm100_ptx.cuh"
+#include "tmem_wide.cuh"
 
 namespace g3 {
 
 // ========================================================= attention kernel
-// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 2-3 idle, warps 4-7 = softmax of head 0, warps 8-11 =
-// softmax of head 1 (when two heads share the K/V tiles).
-constexpr int kAttnThreads = 384;
+// Warp roles (640 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
+// TMEM owner, warps 2-3 idle, warps 4-11 = softmax of head 0, warps 12-19 =
+// softmax of head 1 (when two heads share the K/V tiles): two warps per TMEM
+// lane quarter, each on 16 of its 32 rows.
+constexpr int kAttnThreads = 640;
 constexpr int kSwizzleBlock = 128 * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle column)
 
 template <int D, int HPC>
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int h = 0; h < HPC; ++h) {
       mbar_init(&bars->s_full[h], 1);
-      mbar_init(&bars->p_full[h], 128);
+      mbar_init(&bars->p_full[h], 256);
       mbar_init(&bars->o_full[h], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -114,11 +116,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  // Producer / MMA warpgroup gives registers to the two softmax warpgroups
-  // (128 x 56 + 256 x 224 = 384 x 168, the launch's register budget).  Each
-  // role runs inside the branch that set its register count.
   if (warp < 4) {
-    setmaxnreg_dec<56>();
    if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -223,115 +221,154 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
    }
   } else {
-    setmaxnreg_inc<224>();
-   if (warp < 4 + 4 * HPC) {
-    // ------------------------------------------------------------- softmax
-    const int h = (warp - 4) >> 2;
-    const int lane_base = (warp & 3) * 32;
-    const int row_in = lane_base + lane;
-    const int row = r0 + row_in;
-    const bool valid = row < p.S;
-    const int lo_i = valid ? p.lo[rowbase + row] : 1;
-    const int hi_i = valid ? p.hi[rowbase + row] : 0;
-    const uint32_t t_lane = tmem + ((uint32_t)lane_base << 16);
-    const uint32_t s_col = h * 128;
-    const uint32_t o_col = HPC * 128 + h * D;
-    const float sc = p.scale_log2;
+    const int h = (warp - 4) >> 3;  // query head of the pair
+    if (h < HPC) {
+      // ----------------------------------------------------------- softmax
+      // Warp (quarter q = warp % 4, half s) owns TMEM lanes 32q + 16s .. +15;
+      // thread t holds rows ra = t/4 and rb = t/4 + 8 of that slice and, in
+      // every 8-column chunk k, columns 8k + 2(t%4) and 8k + 2(t%4) + 1; the
+      // four threads t%4 = 0..3 of a row combine their partials by shuffles.
+      const int lane_base = (warp & 3) * 32 + (((warp - 4) >> 2) & 1) * 16;
+      const int m4 = lane & 3;
+      const int ra = lane_base + (lane >> 2), rb = ra + 8;
+      const bool valid_a = r0 + ra < p.S, valid_b = r0 + rb < p.S;
+      const int lo_a = valid_a ? p.lo[rowbase + r0 + ra] : 1, hi_a = valid_a ? p.hi[rowbase + r0 + ra] : 0;
+      const int lo_b = valid_b ? p.lo[rowbase + r0 + rb] : 1, hi_b = valid_b ? p.hi[rowbase + r0 + rb] : 0;
+      const uint32_t t_lane = tmem + ((uint32_t)lane_base << 16);
+      const uint32_t s_col = h * 128;
+      const uint32_t o_col = HPC * 128 + h * D;
+      const float sc = p.scale_log2;
 
-    float m_ref = -INFINITY, l_sum = 0.f;
-    bool ok = true;
-    for (int t = 0; t < n_tiles; ++t) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], t & 1, abort, p.err, 20));
-      if (!ok) break;
-      tc_fence_after();
-      float sv[128];
+      float mref_a = -INFINITY, mref_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+      bool ok = true;
+      for (int t = 0; t < n_tiles; ++t) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], t & 1, abort, p.err, 20));
+        if (!ok) break;
+        tc_fence_after();
+        float sv[64];
+        tmem_ld_16x256b_x16(t_lane + s_col, sv);
+        tmem_wait_ld();
+        const int tile0 = (t_begin + t) * 128;
+        const bool full = tile0 >= lo_last && tile0 + 127 <= hi_first;
+        if (!full) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + s_col + c * 32, sv + c * 32);
-      tmem_wait_ld();
-      const int kv0 = (t_begin + t) * 128;
-      const bool full = kv0 >= lo_last && kv0 + 127 <= hi_first;
-      if (!full) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int j = kv0 + c;
-          if (j < lo_i || j > hi_i) sv[c] = -INFINITY;
+          for (int k = 0; k < 16; ++k) {
+            const int col = tile0 + 8 * k + 2 * m4;
+            if (col < lo_a || col > hi_a) sv[4 * k] = -INFINITY;
+            if (col + 1 < lo_a || col + 1 > hi_a) sv[4 * k + 1] = -INFINITY;
+            if (col < lo_b || col > hi_b) sv[4 * k + 2] = -INFINITY;
+            if (col + 1 < lo_b || col + 1 > hi_b) sv[4 * k + 3] = -INFINITY;
+          }
         }
-      }
-      float mx0 = fmax3(sv[0], sv[1], sv[2]), mx1 = fmax3(sv[3], sv[4], sv[5]);
+        float mxa = fmax3(sv[0], sv[1], sv[4]), mxb = fmax3(sv[2], sv[3], sv[6]);
+        mxa = fmax3(mxa, sv[5], sv[8]);
+        mxb = fmax3(mxb, sv[7], sv[10]);
 #pragma unroll
-      for (int c = 6; c < 126; c += 4) {
-        mx0 = fmax3(mx0, sv[c], sv[c + 1]);
-        mx1 = fmax3(mx1, sv[c + 2], sv[c + 3]);
-      }
-      const float mx = fmax3(fmax3(mx0, mx1, sv[126]), sv[127], sv[127]);
-      const float m_new = fmaxf(m_ref, mx * sc);
-      const bool first = (m_ref == -INFINITY);
-      const bool need = !first && (m_new > m_ref + 8.f);
-      if (first) m_ref = m_new;
-      if (__any_sync(0xffffffffu, need)) {
-        float alpha = 1.f;
-        if (!first) {
-          alpha = ex2_approx(m_ref - m_new);
-          m_ref = m_new;
+        for (int k = 2; k < 16; ++k) {
+          if (k > 2) {
+            mxa = fmax3(mxa, sv[4 * k], sv[4 * k + 1]);
+            mxb = fmax3(mxb, sv[4 * k + 2], sv[4 * k + 3]);
+          } else {
+            mxa = fmaxf(mxa, sv[9]);
+            mxb = fmaxf(mxb, sv[11]);
+          }
         }
-        l_sum *= alpha;
+        mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+        mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+        mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+        mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+        const float mna = fmaxf(mref_a, mxa * sc), mnb = fmaxf(mref_b, mxb * sc);
+        const bool first_a = (mref_a == -INFINITY), first_b = (mref_b == -INFINITY);
+        const bool need = (!first_a && mna > mref_a + 8.f) || (!first_b && mnb > mref_b + 8.f);
+        if (first_a) mref_a = mna;
+        if (first_b) mref_b = mnb;
+        const bool rescale = __any_sync(0xffffffffu, need);
+        float alpha_a = 1.f, alpha_b = 1.f;
+        if (rescale) {
+          if (!first_a) {
+            alpha_a = ex2_approx(mref_a - mna);
+            mref_a = mna;
+          }
+          if (!first_b) {
+            alpha_b = ex2_approx(mref_b - mnb);
+            mref_b = mnb;
+          }
+          l_a *= alpha_a;
+          l_b *= alpha_b;
+        }
+        const float mua = (mref_a == -INFINITY) ? 0.f : mref_a;
+        const float mub = (mref_b == -INFINITY) ? 0.f : mref_b;
+        float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int k = 0; k < 16; ++k) {
+          float x0, x1, x2, x3;
+          ffma2_bcast(sv[4 * k], sv[4 * k + 1], sc, -mua, x0, x1);
+          ffma2_bcast(sv[4 * k + 2], sv[4 * k + 3], sc, -mub, x2, x3);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+          fadd2(sa0, sa1, p0, p1);
+          fadd2(sb0, sb1, p2, p3);
+          pk[2 * k] = pack_bf16x2(p0, p1);
+          pk[2 * k + 1] = pack_bf16x2(p2, p3);
+        }
+        l_a += sa0 + sa1;
+        l_b += sb0 + sb1;
+        // P (bf16 pairs) over the first 64 columns of this head's S region.
+        tmem_st_16x128b_x16(t_lane + s_col, pk);
+        if (rescale) {
+          // O is idle here: the previous P·V has completed (it was issued
+          // before this tile's S) and the next one waits for p_full.
+#pragma unroll
+          for (int q = 0; q < D / 64; ++q) {
+            float o[32];
+            tmem_ld_16x256b_x8(t_lane + o_col + q * 64, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              o[4 * k] *= alpha_a;
+              o[4 * k + 1] *= alpha_a;
+              o[4 * k + 2] *= alpha_b;
+              o[4 * k + 3] *= alpha_b;
+            }
+            tmem_st_16x256b_x8(t_lane + o_col + q * 64, reinterpret_cast<uint32_t*>(o));
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[h]);
+      }
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[h], 0, abort, p.err, 21));
+      if (ok) {
+        tc_fence_after();
+        const float inv_a = 1.f / l_a, inv_b = 1.f / l_b;
+        const int hq = h0 + h;
+        __nv_bfloat16* da = p.out + ((rowbase + r0 + ra) * p.Hq + hq) * D + 2 * m4;
+        __nv_bfloat16* db = p.out + ((rowbase + r0 + rb) * p.Hq + hq) * D + 2 * m4;
+#pragma unroll
+        for (int q = 0; q < D / 64; ++q) {
           float o[32];
-          tmem_ld32(t_lane + o_col + c * 32, o);
+          tmem_ld_16x256b_x8(t_lane + o_col + q * 64, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(t_lane + o_col + c * 32, reinterpret_cast<uint32_t*>(o));
+          for (int k = 0; k < 8; ++k) {
+            const int c = q * 64 + 8 * k;
+            if (valid_a) *reinterpret_cast<uint32_t*>(da + c) = pack_bf16x2(o[4 * k] * inv_a, o[4 * k + 1] * inv_a);
+            if (valid_b)
+              *reinterpret_cast<uint32_t*>(db + c) = pack_bf16x2(o[4 * k + 2] * inv_b, o[4 * k + 3] * inv_b);
+          }
+        }
+        if (m4 == 0 && p.lse != nullptr) {
+          const size_t lrow = ((size_t)b * p.Hq + hq) * p.S + r0;
+          if (valid_a) p.lse[lrow + ra] = (mref_a + log2f(l_a)) * 0.69314718055994530942f;
+          if (valid_b) p.lse[lrow + rb] = (mref_b + log2f(l_b)) * 0.69314718055994530942f;
         }
       }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // Exponentials two at a time (one f16x2 exp-unit operation per pair),
-      // scaling and sums as packed fp32x2 operations, two partial sum pairs.
-      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float x0, x1, p0, p1;
-        ffma2_bcast(sv[2 * c], sv[2 * c + 1], sc, -m_use, x0, x1);
-        ex2_pair_f16(x0, x1, p0, p1);
-        if (c & 1) {
-          fadd2(sb0, sb1, p0, p1);
-        } else {
-          fadd2(sa0, sa1, p0, p1);
-        }
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      l_sum += (sa0 + sa1) + (sb0 + sb1);
-      tmem_st32(t_lane + s_col, pk);
-      tmem_st32(t_lane + s_col + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[h]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[h], 0, abort, p.err, 21));
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = 1.f / l_sum;
-      const int hq = h0 + h;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + ((rowbase + row) * p.Hq + hq) * D);
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(t_lane + o_col + c * 32, o);
-        tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
-        if (valid) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[c * 4 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
-      }
-      if (valid && p.lse != nullptr)
-        p.lse[((size_t)b * p.Hq + hq) * p.S + row] = (m_ref + log2f(l_sum)) * 0.69314718055994530942f;
-    }
-   }
   }
 
   tc_fence_before();
@@ -353,9 +390,13 @@ static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, con
                                  const CUtensorMap& tv, cudaStream_t st) {
   using L = AttnLayout<D, HPC>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(prefill_attention_kernel<D, HPC>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-  if (e != cudaSuccess) return e;
+  static bool configured = false;  // the attribute belongs to the function; set it once
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(prefill_attention_kernel<D, HPC>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hkv * p.n_groups;
   prefill_attention_kernel<D, HPC><<<grid, kAttnThreads, L::kAlloc, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
