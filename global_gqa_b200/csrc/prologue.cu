@@ -7,8 +7,10 @@
 //                 of the image spans.
 //   qk_norm_rope: bandwidth-bound pass over every (token, head) row of q and k.
 //                 One warp per token: the token's cos/sin are loaded once into
-//                 registers and serve all of its Hq + Hkv rows; eight row steps
-//                 of 8-byte loads per lane are in flight; no block-wide sync.
+//                 registers and serve all of its Hq + Hkv rows; each lane
+//                 holds 8 features of each half of a row (16-byte accesses,
+//                 rotation partners in the same lane), four row steps in
+//                 flight; no block-wide sync.
 //
 // Norm (Gemma 3 Technical Report, section 2; eps and dim from the q_norm /
 // k_norm lines of "Gemma explained: what's new in Gemma 3"): x / sqrt(mean(x^2)
@@ -34,7 +36,7 @@ namespace g3 {
 
 constexpr int kTableThreads = 256;
 constexpr int kRowThreads = 256;  // 8 warps, one token each at a time
-constexpr int kRowUnroll = 8;     // row steps in flight per warp
+constexpr int kRowUnroll = 4;     // row steps in flight per warp
 
 template <int D>
 __global__ void __launch_bounds__(kTableThreads) rope_table_kernel(PrologueParams p) {
@@ -91,89 +93,101 @@ __device__ __forceinline__ uint2 pack4_bf16(const float* f) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kRowThreads, 3) qk_norm_rope_kernel(PrologueParams p) {
+__global__ void __launch_bounds__(kRowThreads, 2) qk_norm_rope_kernel(PrologueParams p) {
   constexpr int H2 = D / 2;
-  constexpr int LPR = D / 8;     // lanes per row: each holds 4 features of each half
+  constexpr int LPR = D / 16;    // lanes per row: each holds 8 features of each half
   constexpr int RPW = 32 / LPR;  // rows per warp step
   const int lane = threadIdx.x & 31;
   const int li = lane % LPR, sub = lane / LPR;
-  const int d1 = li * 4;  // this lane: features d1..d1+3 and H2+d1..H2+d1+3
+  const int d1 = li * 8;  // this lane: features d1..d1+7 and H2+d1..H2+d1+7 (rotation partners)
   const int heads = p.Hq + p.Hkv;
   const int n_tokens = p.B * p.S;
   const int warps_total = gridDim.x * (kRowThreads / 32);
+  float gq[16], gk[16];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    gq[e] = p.q_gamma[d1 + e];
+    gq[8 + e] = p.q_gamma[H2 + d1 + e];
+    gk[e] = p.k_gamma[d1 + e];
+    gk[8 + e] = p.k_gamma[H2 + d1 + e];
+  }
 
   for (int bt = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); bt < n_tokens; bt += warps_total) {
     const float4* tab = reinterpret_cast<const float4*>(p.rope_table + (size_t)bt * H2 + d1);
-    const float4 cs0 = __ldg(tab), cs1 = __ldg(tab + 1);
-    const float c[4] = {cs0.x, cs0.z, cs1.x, cs1.z};
-    const float s[4] = {cs0.y, cs0.w, cs1.y, cs1.w};
+    float c[8], s[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldg(tab + i);
+      c[2 * i] = v.x;
+      s[2 * i] = v.y;
+      c[2 * i + 1] = v.z;
+      s[2 * i + 1] = v.w;
+    }
     const __nv_bfloat16* qrow = p.q + (size_t)bt * p.Hq * D;
     const __nv_bfloat16* krow = p.k + (size_t)bt * p.Hkv * D;
 
     for (int h0 = 0; h0 < heads; h0 += RPW * kRowUnroll) {
-      uint2 xa[kRowUnroll], xb[kRowUnroll];
+      uint4 xa[kRowUnroll], xb[kRowUnroll];
 #pragma unroll
       for (int u = 0; u < kRowUnroll; ++u) {
         const int h = h0 + u * RPW + sub;
         if (h < heads) {
           const __nv_bfloat16* src = h < p.Hq ? qrow + h * D : krow + (h - p.Hq) * D;
-          xa[u] = __ldg(reinterpret_cast<const uint2*>(src + d1));
-          xb[u] = __ldg(reinterpret_cast<const uint2*>(src + H2 + d1));
+          xa[u] = __ldg(reinterpret_cast<const uint4*>(src + d1));
+          xb[u] = __ldg(reinterpret_cast<const uint4*>(src + H2 + d1));
         } else {
-          xa[u] = xb[u] = make_uint2(0u, 0u);
+          xa[u] = xb[u] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
 #pragma unroll
       for (int u = 0; u < kRowUnroll; ++u) {
-        float x[8];
-        unpack4_bf16(xa[u], x);
-        unpack4_bf16(xb[u], x + 4);
+        float x[16];
+        unpack4_bf16(make_uint2(xa[u].x, xa[u].y), x);
+        unpack4_bf16(make_uint2(xa[u].z, xa[u].w), x + 4);
+        unpack4_bf16(make_uint2(xb[u].x, xb[u].y), x + 8);
+        unpack4_bf16(make_uint2(xb[u].z, xb[u].w), x + 12);
         float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+        for (int e = 0; e < 16; ++e) ss = fmaf(x[e], x[e], ss);
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         const int h = h0 + u * RPW + sub;
         if (h >= heads) continue;
         const bool is_q = h < p.Hq;
         const float rinv = rsqrtf(ss * (1.0f / D) + 1e-6f);
-        const float* gam = is_q ? p.q_gamma : p.k_gamma;
-        const float4 ga = __ldg(reinterpret_cast<const float4*>(gam + d1));
-        const float4 gb = __ldg(reinterpret_cast<const float4*>(gam + H2 + d1));
-        const float g1[4] = {ga.x, ga.y, ga.z, ga.w};
-        const float g2[4] = {gb.x, gb.y, gb.z, gb.w};
-        float o[8];
+        const float* g = is_q ? gq : gk;
+        float o[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float y1 = x[e] * rinv * g1[e];
-          const float y2 = x[4 + e] * rinv * g2[e];
+        for (int e = 0; e < 8; ++e) {
+          const float y1 = x[e] * rinv * g[e];
+          const float y2 = x[8 + e] * rinv * g[8 + e];
           o[e] = y1 * c[e] - y2 * s[e];
-          o[4 + e] = y1 * s[e] + y2 * c[e];
+          o[8 + e] = y1 * s[e] + y2 * c[e];
         }
-        const uint2 lo4 = pack4_bf16(o), hi4 = pack4_bf16(o + 4);
+        const uint2 a0 = pack4_bf16(o), a1 = pack4_bf16(o + 4), b0 = pack4_bf16(o + 8), b1 = pack4_bf16(o + 12);
+        const uint4 lo8 = make_uint4(a0.x, a0.y, a1.x, a1.y), hi8 = make_uint4(b0.x, b0.y, b1.x, b1.y);
         if (is_q) {
           __nv_bfloat16* dst = p.q_hat + ((size_t)bt * p.Hq + h) * D;
-          *reinterpret_cast<uint2*>(dst + d1) = lo4;
-          *reinterpret_cast<uint2*>(dst + H2 + d1) = hi4;
+          *reinterpret_cast<uint4*>(dst + d1) = lo8;
+          *reinterpret_cast<uint4*>(dst + H2 + d1) = hi8;
         } else {
           const int kh = h - p.Hq;
           const size_t row = (size_t)bt * p.Hkv + kh;
           __nv_bfloat16* dst = p.k_hat + row * D;
-          *reinterpret_cast<uint2*>(dst + d1) = lo4;
-          *reinterpret_cast<uint2*>(dst + H2 + d1) = hi4;
+          *reinterpret_cast<uint4*>(dst + d1) = lo8;
+          *reinterpret_cast<uint4*>(dst + H2 + d1) = hi8;
           if (p.k_cache != nullptr) {
             const int b = bt / p.S, t = bt % p.S;
             const bool write = (p.kind == 1) ? (t < p.cache_cap) : (t >= p.S - p.cache_cap);
             if (write) {
               const int slot = (p.kind == 1) ? t : t % p.cache_cap;
               const size_t crow = ((size_t)b * p.Hkv + kh) * p.cache_cap + slot;
-              *reinterpret_cast<uint2*>(p.k_cache + crow * D + d1) = lo4;
-              *reinterpret_cast<uint2*>(p.k_cache + crow * D + H2 + d1) = hi4;
+              *reinterpret_cast<uint4*>(p.k_cache + crow * D + d1) = lo8;
+              *reinterpret_cast<uint4*>(p.k_cache + crow * D + H2 + d1) = hi8;
               const __nv_bfloat16* vsrc = p.v + row * D;
-              *reinterpret_cast<uint2*>(p.v_cache + crow * D + d1) =
-                  __ldg(reinterpret_cast<const uint2*>(vsrc + d1));
-              *reinterpret_cast<uint2*>(p.v_cache + crow * D + H2 + d1) =
-                  __ldg(reinterpret_cast<const uint2*>(vsrc + H2 + d1));
+              *reinterpret_cast<uint4*>(p.v_cache + crow * D + d1) = __ldg(reinterpret_cast<const uint4*>(vsrc + d1));
+              *reinterpret_cast<uint4*>(p.v_cache + crow * D + H2 + d1) =
+                  __ldg(reinterpret_cast<const uint4*>(vsrc + H2 + d1));
             }
           }
         }
