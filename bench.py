@@ -255,6 +255,26 @@ def run_gpu(args, rank, world, local_rank):
     kernels = {k: {"launches": v[0], "ms": v[1], "share": v[1] / max(sum(x[1] for x in trace.values()), 1e-9)}
                for k, v in trace.items()}
 
+    # ---- per layer kind (outside the timed region): one local and the global layer
+    layer_kinds = {}
+    for li in (0, len(blk) - 1):
+        L, x = layers[li]
+        f = metrics.layer_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, L.kind, L.window)
+        g3.trace_collect()
+        barrier()
+        g3.trace_enable(True)
+        for _ in range(max(args.steps, 5)):
+            g3.prefill(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind, L.window,
+                       L.rope_base, L.interp, x["spans"], out=x["out"], ws=ws, stream=stream)
+        barrier()
+        g3.trace_enable(False)
+        tr = g3.trace_collect()
+        na, ma = tr.get("prefill_attention", (1, 0.0))
+        npro, mpro = tr.get("prefill_prologue", (1, 0.0))
+        layer_kinds["local" if L.kind == 0 else "global"] = {
+            "flops": f, "attention_us": 1e3 * ma / na, "attention_tflops": f / (ma / na * 1e-3) / 1e12,
+            "prologue_us": 1e3 * mpro / npro}
+
     # ---- end to end through the public API from pinned host memory
     host = []
     for L, x in layers:
@@ -303,6 +323,7 @@ def run_gpu(args, rank, world, local_rank):
                    "parallelism": f"independent replicas x{world}"},
         "roofline": roofline,
         "kernels": kernels,
+        "layer_kinds": layer_kinds,
         "gpu_launches": sum(v[0] for v in trace.values()),
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
