@@ -212,7 +212,11 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "prefill: head_dim %d not built (64, 128)", D);
   if ((size_t)B * S * Hq * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "prefill: problem too large");
   const int G = Hq / Hkv;
-  const int hpc = (G % 2 == 0) ? 2 : 1;
+  // Heads per attention CTA.  Two heads of a kv group share each K/V tile
+  // (one CTA per SM); sliding-window layers visit few tiles per query tile, so
+  // there one-head CTAs, two per SM, hide each other's start and epilogue and
+  // run faster.
+  const int hpc = (G % 2 == 0 && layer_kind == G3_LAYER_GLOBAL) ? 2 : 1;
   const long long n_qtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
   if (n_qtiles * B * Hkv * (G / hpc) > 0x7fffffffLL) return fail(G3_ERR_UNSUPPORTED, "prefill: grid too large");
 

@@ -29,16 +29,25 @@
 namespace g3 {
 
 // ========================================================= attention kernel
-// Warp roles (640 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 2-3 idle, warps 4-11 = softmax of head 0, warps 12-19 =
-// softmax of head 1 (when two heads share the K/V tiles): two warps per TMEM
-// lane quarter, each on 16 of its 32 rows.
-constexpr int kAttnThreads = 640;
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and TMEM owner, then
+// eight softmax warps per query head (warps 4-11 and 12-19 when two heads share
+// the K/V tiles, warps 2-9 for one head): two warps per TMEM lane quarter,
+// each on 16 of its 32 rows.
+template <int HPC>
+struct AttnRoles {
+  // Two heads: 640 threads, one CTA per SM.  One head: 320 threads (warp 0
+  // producer, warp 1 MMA, warps 2-9 softmax) and two CTAs per SM, so one
+  // CTA's start and epilogue overlap the other's main loop.
+  static constexpr int kFirstSoftmaxWarp = (HPC == 2) ? 4 : 2;
+  static constexpr int kThreads = (kFirstSoftmaxWarp + 8 * HPC) * 32;
+  static constexpr int kMinBlocks = (HPC == 2) ? 1 : 2;
+};
 constexpr int kSwizzleBlock = 128 * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle column)
 
 template <int D, int HPC>
 struct AttnLayout {
-  static constexpr int kStages = (D == 64) ? 3 : 2;
+  // K/V ring depth; one-head CTAs keep two CTAs' shared memory within one SM.
+  static constexpr int kStages = (HPC == 2) ? (D == 64 ? 3 : 2) : (D == 64 ? 2 : 1);
   static constexpr int kTile = 128 * D * 2;  // bytes of one 128-row tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + HPC * kTile;
@@ -59,7 +68,7 @@ struct AttnBarriers {
 };
 
 template <int D, int HPC>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMinBlocks)
     prefill_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
   using L = AttnLayout<D, HPC>;
@@ -116,7 +125,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 4) {
+  constexpr int SW0 = AttnRoles<HPC>::kFirstSoftmaxWarp;
+  if (warp < SW0) {
    if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -221,14 +231,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
    }
   } else {
-    const int h = (warp - 4) >> 3;  // query head of the pair
+    const int h = (warp - SW0) >> 3;  // query head of the pair
     if (h < HPC) {
       // ----------------------------------------------------------- softmax
       // Warp (quarter q = warp % 4, half s) owns TMEM lanes 32q + 16s .. +15;
       // thread t holds rows ra = t/4 and rb = t/4 + 8 of that slice and, in
       // every 8-column chunk k, columns 8k + 2(t%4) and 8k + 2(t%4) + 1; the
       // four threads t%4 = 0..3 of a row combine their partials by shuffles.
-      const int lane_base = (warp & 3) * 32 + (((warp - 4) >> 2) & 1) * 16;
+      const int lane_base = (warp & 3) * 32 + (((warp - SW0) >> 2) & 1) * 16;
       const int m4 = lane & 3;
       const int ra = lane_base + (lane >> 2), rb = ra + 8;
       const bool valid_a = r0 + ra < p.S, valid_b = r0 + rb < p.S;
@@ -398,7 +408,7 @@ static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, con
     configured = true;
   }
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hkv * p.n_groups;
-  prefill_attention_kernel<D, HPC><<<grid, kAttnThreads, L::kAlloc, st>>>(tq, tk, tv, p);
+  prefill_attention_kernel<D, HPC><<<grid, AttnRoles<HPC>::kThreads, L::kAlloc, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
