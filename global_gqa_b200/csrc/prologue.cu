@@ -9,8 +9,9 @@
 //                 One warp per token: the token's cos/sin are loaded once into
 //                 registers and serve all of its Hq + Hkv rows; each lane
 //                 holds 8 features of each half of a row (16-byte accesses,
-//                 rotation partners in the same lane), four row steps in
-//                 flight; no block-wide sync.
+//                 rotation partners in the same lane), two row steps in
+//                 flight per warp and 32 warps per SM; the gains are read
+//                 from shared memory to keep registers free.
 //
 // Norm (Gemma 3 Technical Report, section 2; eps and dim from the q_norm /
 // k_norm lines of "Gemma explained: what's new in Gemma 3"): x / sqrt(mean(x^2)
@@ -36,18 +37,21 @@ namespace g3 {
 
 constexpr int kTableThreads = 256;
 constexpr int kRowThreads = 256;  // 8 warps, one token each at a time
-constexpr int kRowUnroll = 4;     // row steps in flight per warp
+constexpr int kRowUnroll = 2;     // row steps in flight per warp (32 warps per SM)
 
 template <int D>
 __global__ void __launch_bounds__(kTableThreads) rope_table_kernel(PrologueParams p) {
   constexpr int H2 = D / 2;
+  __shared__ double inv_freq_s[H2];
+  if (threadIdx.x < H2) inv_freq_s[threadIdx.x] = p.inv_freq[threadIdx.x];
+  __syncthreads();
   const size_t idx = (size_t)blockIdx.x * kTableThreads + threadIdx.x;
   const size_t total = (size_t)p.B * p.S * H2;
   if (idx >= total) return;
   const size_t bt = idx / H2;
   const int f = (int)(idx % H2);
   const int b = (int)(bt / p.S), t = (int)(bt % p.S);
-  const double theta = (double)p.positions[bt] / p.interp * p.inv_freq[f];
+  const double theta = (double)p.positions[bt] / p.interp * inv_freq_s[f];
   double sd, cd;
   sincos(theta, &sd, &cd);
   p.rope_table[idx] = make_float2((float)cd, (float)sd);
@@ -93,7 +97,7 @@ __device__ __forceinline__ uint2 pack4_bf16(const float* f) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kRowThreads, 2) qk_norm_rope_kernel(PrologueParams p) {
+__global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(PrologueParams p) {
   constexpr int H2 = D / 2;
   constexpr int LPR = D / 16;    // lanes per row: each holds 8 features of each half
   constexpr int RPW = 32 / LPR;  // rows per warp step
@@ -103,14 +107,9 @@ __global__ void __launch_bounds__(kRowThreads, 2) qk_norm_rope_kernel(ProloguePa
   const int heads = p.Hq + p.Hkv;
   const int n_tokens = p.B * p.S;
   const int warps_total = gridDim.x * (kRowThreads / 32);
-  float gq[16], gk[16];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    gq[e] = p.q_gamma[d1 + e];
-    gq[8 + e] = p.q_gamma[H2 + d1 + e];
-    gk[e] = p.k_gamma[d1 + e];
-    gk[8 + e] = p.k_gamma[H2 + d1 + e];
-  }
+  __shared__ __align__(16) float gam[2 * D];  // q gain, then k gain
+  for (int i = threadIdx.x; i < 2 * D; i += kRowThreads) gam[i] = i < D ? p.q_gamma[i] : p.k_gamma[i - D];
+  __syncthreads();
 
   for (int bt = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); bt < n_tokens; bt += warps_total) {
     const float4* tab = reinterpret_cast<const float4*>(p.rope_table + (size_t)bt * H2 + d1);
@@ -155,7 +154,12 @@ __global__ void __launch_bounds__(kRowThreads, 2) qk_norm_rope_kernel(ProloguePa
         if (h >= heads) continue;
         const bool is_q = h < p.Hq;
         const float rinv = rsqrtf(ss * (1.0f / D) + 1e-6f);
-        const float* g = is_q ? gq : gk;
+        const float* gs = gam + (is_q ? 0 : D);
+        float g[16];
+        *reinterpret_cast<float4*>(g) = *reinterpret_cast<const float4*>(gs + d1);
+        *reinterpret_cast<float4*>(g + 4) = *reinterpret_cast<const float4*>(gs + d1 + 4);
+        *reinterpret_cast<float4*>(g + 8) = *reinterpret_cast<const float4*>(gs + H2 + d1);
+        *reinterpret_cast<float4*>(g + 12) = *reinterpret_cast<const float4*>(gs + H2 + d1 + 4);
         float o[16];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
