@@ -144,7 +144,7 @@ bool decode_ws(int B, int Hq, int Hkv, int D, int max_len, DecodeWs* w) {
   return true;
 }
 
-bool supported_d(int D) { return D == 64 || D == 128; }
+bool supported_d(int D) { return D == 64 || D == 128 || D == 256; }
 
 }  // namespace
 
@@ -209,14 +209,15 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
     if (layer_kind == G3_LAYER_LOCAL && cache_capacity != window)
       return fail(G3_ERR_INVALID_ARG, "prefill: local ring capacity %d != window %d", cache_capacity, window);
   }
-  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "prefill: head_dim %d not built (64, 128)", D);
+  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "prefill: head_dim %d not built (64, 128, 256)", D);
   if ((size_t)B * S * Hq * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "prefill: problem too large");
   const int G = Hq / Hkv;
   // Heads per attention CTA.  Two heads of a kv group share each K/V tile
   // (one CTA per SM); sliding-window layers visit few tiles per query tile, so
   // there one-head CTAs, two per SM, hide each other's start and epilogue and
   // run faster.
-  const int hpc = (G % 2 == 0 && layer_kind == G3_LAYER_GLOBAL) ? 2 : 1;
+  // (At D = 256 one head's S and O already take 384 of the 512 TMEM columns.)
+  const int hpc = (G % 2 == 0 && layer_kind == G3_LAYER_GLOBAL && D <= 128) ? 2 : 1;
   const long long n_qtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
   if (n_qtiles * B * Hkv * (G / hpc) > 0x7fffffffLL) return fail(G3_ERR_UNSUPPORTED, "prefill: grid too large");
 
@@ -308,7 +309,7 @@ g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new, con
     return fail(G3_ERR_INVALID_ARG, "decode: bad interp_factor");
   if (!aligned16(k_cache) || !aligned16(v_cache))
     return fail(G3_ERR_INVALID_ARG, "decode: caches must be 16-byte aligned");
-  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "decode: head_dim %d not built (64, 128)", D);
+  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "decode: head_dim %d not built (64, 128, 256)", D);
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4) return fail(G3_ERR_UNSUPPORTED, "decode: group size %d not built (1, 2, 4)", G);
   if ((size_t)B * Hkv * cache_capacity * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "decode: cache too large");

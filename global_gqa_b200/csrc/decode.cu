@@ -290,6 +290,8 @@ cudaError_t launch_decode_prologue(const DecodeParams& p, int D, cudaStream_t st
     decode_prologue_kernel<128><<<p.B, kDecPrologueThreads, 0, st>>>(p);
   else if (D == 64)
     decode_prologue_kernel<64><<<p.B, kDecPrologueThreads, 0, st>>>(p);
+  else if (D == 256)
+    decode_prologue_kernel<256><<<p.B, kDecPrologueThreads, 0, st>>>(p);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
@@ -311,6 +313,7 @@ cudaError_t launch_decode_split(const DecodeParams& p, int D, int grid_chunks, c
   if (grid_chunks < 1 || grid_chunks > p.n_chunks) return cudaErrorInvalidValue;
   if (D == 128) return launch_split_d<128>(p, grid_chunks, st);
   if (D == 64) return launch_split_d<64>(p, grid_chunks, st);
+  if (D == 256) return launch_split_d<256>(p, grid_chunks, st);
   return cudaErrorInvalidValue;
 }
 
@@ -319,6 +322,8 @@ cudaError_t launch_decode_combine(const DecodeParams& p, int D, cudaStream_t st)
     decode_combine_kernel<128><<<p.B * p.Hq, 128, 0, st>>>(p);
   else if (D == 64)
     decode_combine_kernel<64><<<p.B * p.Hq, 64, 0, st>>>(p);
+  else if (D == 256)
+    decode_combine_kernel<256><<<p.B * p.Hq, 256, 0, st>>>(p);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

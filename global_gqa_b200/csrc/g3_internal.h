@@ -29,7 +29,7 @@ struct PrologueParams {
   int window;
   double rope_base;
   double interp;
-  double inv_freq[64];   // base^(-2f/D), f < D/2, computed on the host in double
+  double inv_freq[128];  // base^(-2f/D), f < D/2 (D <= 256), computed on the host in double
   __nv_bfloat16* q_hat;  // [B,S,Hq,D]
   __nv_bfloat16* k_hat;  // [B,S,Hkv,D]
   int32_t* lo;           // [B,S] first visible key of each row

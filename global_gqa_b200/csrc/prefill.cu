@@ -391,6 +391,7 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
 }
 
 size_t prefill_attention_smem_bytes(int D, int hpc) {
+  if (D == 256) return AttnLayout<256, 1>::kAlloc;
   if (D == 128) return hpc == 2 ? AttnLayout<128, 2>::kAlloc : AttnLayout<128, 1>::kAlloc;
   return hpc == 2 ? AttnLayout<64, 2>::kAlloc : AttnLayout<64, 1>::kAlloc;
 }
@@ -414,6 +415,7 @@ static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, con
 
 cudaError_t launch_prefill_attention(const AttnParams& p, int D, int hpc, const CUtensorMap& tq,
                                      const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+  if (D == 256 && hpc == 1) return launch_attn_t<256, 1>(p, tq, tk, tv, st);
   if (D == 128 && hpc == 2) return launch_attn_t<128, 2>(p, tq, tk, tv, st);
   if (D == 128 && hpc == 1) return launch_attn_t<128, 1>(p, tq, tk, tv, st);
   if (D == 64 && hpc == 2) return launch_attn_t<64, 2>(p, tq, tk, tv, st);

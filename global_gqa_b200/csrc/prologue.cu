@@ -212,6 +212,9 @@ cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t
   } else if (D == 64) {
     rope_table_kernel<64><<<table_blocks, kTableThreads, 0, st>>>(p);
     qk_norm_rope_kernel<64><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
+  } else if (D == 256) {
+    rope_table_kernel<256><<<table_blocks, kTableThreads, 0, st>>>(p);
+    qk_norm_rope_kernel<256><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
   } else {
     return cudaErrorInvalidValue;
   }

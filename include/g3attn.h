@@ -80,7 +80,7 @@ size_t g3attn_prefill_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t H
  *   rope_base  > 0;  interp_factor > 0 (positions are divided by it)
  *   image_spans int32 [B, n_spans, 2] half-open [start, end) per sequence,
  *              sorted, disjoint, 0 <= start < end <= S; NULL iff n_spans == 0
- *   B, S, Hq, Hkv, D   S >= 1, Hq % Hkv == 0, D in {64, 128}
+ *   B, S, Hq, Hkv, D   S >= 1, Hq % Hkv == 0, D in {64, 128, 256}
  *   out        bf16 [B, S, Hq, D]
  *   lse        optional fp32 [B, Hq, S]: natural-log sum of exp of the scaled
  *              scores of each row (NULL to skip)

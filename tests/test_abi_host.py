@@ -66,7 +66,7 @@ def _prefill(lib, **kw):
     (dict(base=float("inf")), 1), (dict(interp=0.0), 1), (dict(n_spans=2), 1),
     (dict(spans=FAKE, n_spans=0), 1), (dict(q=FAKE + 2), 1), (dict(kc=FAKE), 1),
     (dict(kc=FAKE, vc=FAKE, cap=100), 1), (dict(kind=1, kc=FAKE, vc=FAKE, cap=64), 1),
-    (dict(D=96), 2), (dict(D=256), 2), (dict(ws=None), 3), (dict(ws=FAKE * 256 + 16), 3), (dict(wsb=100), 3),
+    (dict(D=96), 2), (dict(D=512), 2), (dict(ws=None), 3), (dict(ws=FAKE * 256 + 16), 3), (dict(wsb=100), 3),
 ])
 def test_prefill_rejects_on_host(lib, kw, code):
     assert _prefill(lib, **kw) == code

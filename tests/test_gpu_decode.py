@@ -72,6 +72,9 @@ SWEEP = [
     (3, 4, 2, 128, [1024, 1025, 2049], O.LOCAL, 1024),
     (2, 8, 2, 128, [3, 100], O.LOCAL, 7),
     (2, 4, 4, 128, [700, 9000], O.LOCAL, 1024),
+    # Gemma 3 1B attention shapes: 4 query heads, 1 kv head, head_dim 256
+    (2, 4, 1, 256, [1, 4097], O.GLOBAL, 512),
+    (3, 4, 1, 256, [511, 1025, 2000], O.LOCAL, 512),
 ]
 
 

@@ -34,6 +34,11 @@ SWEEP = [
     (1, 3000, 4, 2, 64, GLB, 1024, [[1000, 1256]], 1e6, 1.0),
     (1, 777, 4, 4, 64, LOC, 300, None, 1e4, 1.0),
     (1, 2048, 8, 2, 128, GLB, 1024, None, 1e6, 8.0),
+    # Gemma 3 1B attention shapes: 4 query heads, 1 kv head, head_dim 256
+    (1, 300, 4, 1, 256, LOC, 512, [[10, 40], [100, 299]], 1e4, 1.0),
+    (2, 1025, 4, 1, 256, LOC, 1024, [[0, 256]], 1e4, 1.0),
+    (1, 2048, 4, 1, 256, GLB, 1024, None, 1e6, 8.0),
+    (1, 129, 2, 2, 256, GLB, 1024, None, 1e6, 1.0),
 ]
 
 
@@ -141,3 +146,20 @@ def test_bad_spans_reported_on_device():
     run_prefill(xd, LOC, 16, 1e4, 1.0, ws=ws)
     assert g3.check_device_error(ws) == 1
     assert g3.check_device_error(ws) == 0   # read-and-clear
+
+
+@pytest.mark.parametrize("kind", [LOC, GLB], ids=["local", "global"])
+def test_prefill_1b_shapes_32k(kind):
+    """Gemma 3 1B attention shapes (4 query heads, 1 kv head, head_dim 256) at a
+    32K context, on sampled rows of all heads."""
+    B, S, Hq, Hkv, D, W = 1, 32768, 4, 1, 256, 1024
+    base, interp = (1e4, 1.0) if kind == LOC else (1e6, 8.0)
+    xc = inputs.prefill_layer_inputs(B, S, Hq, Hkv, D, seed=0, layer=0 if kind == LOC else 5)
+    xd = to_dev(xc)
+    out, lse = run_prefill(xd, kind, W, base, interp)
+    assert g3.check_device_error(g3.workspace(0, dev())) == 0
+    rows = sampled_rows(S, W, n_random=128)
+    ref, ref_lse = oracle_rows(xc, kind, W, base, interp, rows=rows)
+    idx = torch.as_tensor(rows, device=out.device)
+    assert_close(out[:, idx], ref, what="1B-shaped out")
+    assert_close(lse[:, :, idx], ref_lse, atol=LSE_ATOL, rel_l2=np.inf, what="1B-shaped lse")
