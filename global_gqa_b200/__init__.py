@@ -42,6 +42,10 @@ _SIGS = {
     "g3attn_prefill_workspace_size": (_sz, [_i32] * 5),
     "g3attn_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _i32, _f32, _f32, _vp, _i32,
                                       _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "g3attn_prefill_chunk_workspace_size": (_sz, [_i32] * 6 + [ctypes.c_int, _i32]),
+    "g3attn_prefill_chunk": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_int, _i32,
+                                            _f32, _f32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
+                                            _sz, _vp]),
     "g3attn_decode_workspace_size": (_sz, [_i32] * 5),
     "g3attn_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, ctypes.c_int, _i32,
                                      _f32, _f32, _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
@@ -86,6 +90,11 @@ def _check(status: int, where: str) -> None:
 
 def prefill_workspace_size(B: int, S: int, Hq: int, Hkv: int, D: int) -> int:
     return int(lib().g3attn_prefill_workspace_size(B, S, Hq, Hkv, D))
+
+
+def prefill_chunk_workspace_size(B: int, C: int, Hq: int, Hkv: int, D: int, start: int, layer_kind: int,
+                                 window: int) -> int:
+    return int(lib().g3attn_prefill_chunk_workspace_size(B, C, Hq, Hkv, D, start, int(layer_kind), window))
 
 
 def decode_workspace_size(B: int, Hq: int, Hkv: int, D: int, max_seq_len: int) -> int:
@@ -227,3 +236,50 @@ def trace_collect() -> dict:
     arr = (KernelTrace * 32)()
     n = lib().g3attn_trace_collect(arr, 32)
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}
+
+
+def prefill_chunk(q, k, v, q_gamma, k_gamma, positions, k_cache, v_cache, start: int, layer_kind: int,
+                  window: int, rope_base: float, interp_factor: float, image_spans=None, *, out=None,
+                  return_lse: bool = False, ws=None, stream=None):
+    """The next C tokens of sequences whose first `start` tokens are cached; returns out (and lse).
+
+    q [B,C,Hq,D] bf16, k/v [B,C,Hkv,D] bf16 (raw projections of the chunk),
+    positions int32 [B,C], k_cache/v_cache bf16 [B,Hkv,cap,D] (updated in place),
+    image_spans int32 [B,n,2] in whole-sequence token indices, or None.
+    """
+    torch = _torch()
+    _req(q, "q", torch.bfloat16)
+    B, C, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _req(k, "k", torch.bfloat16, (B, C, Hkv, D))
+    _req(v, "v", torch.bfloat16, (B, C, Hkv, D))
+    _req(q_gamma, "q_gamma", torch.float32, (D,))
+    _req(k_gamma, "k_gamma", torch.float32, (D,))
+    _req(positions, "positions", torch.int32, (B, C))
+    _req(k_cache, "k_cache", torch.bfloat16)
+    _req(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+    if k_cache.dim() != 4 or k_cache.shape[0] != B or k_cache.shape[1] != Hkv or k_cache.shape[3] != D:
+        raise ValueError("k_cache must be [B, Hkv, capacity, D]")
+    cap = int(k_cache.shape[2])
+    n_spans = 0
+    if image_spans is not None:
+        _req(image_spans, "image_spans", torch.int32)
+        if image_spans.dim() != 3 or image_spans.shape[0] != B or image_spans.shape[2] != 2:
+            raise ValueError("image_spans must be [B, n, 2]")
+        n_spans = int(image_spans.shape[1])
+        if n_spans == 0:
+            image_spans = None
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, C, dtype=torch.float32, device=q.device) if return_lse else None
+    need = prefill_chunk_workspace_size(B, C, Hq, Hkv, D, start, layer_kind, window)
+    if need == 0:
+        raise ValueError("invalid sizes for prefill_chunk")
+    wsb = ws if ws is not None else workspace(need, q.device)
+    st = lib().g3attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
+                                    _ptr(k_cache), _ptr(v_cache), cap, int(start), int(layer_kind), int(window),
+                                    float(rope_base), float(interp_factor), _ptr(image_spans), n_spans, B, C, Hq,
+                                    Hkv, D, _ptr(out), _ptr(lse), wsb.data_ptr(), wsb.numel(),
+                                    _stream_ptr(stream, q.device))
+    _check(st, "g3attn_prefill_chunk")
+    return (out, lse) if return_lse else out

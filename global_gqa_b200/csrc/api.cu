@@ -102,6 +102,23 @@ bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int 
   return r == CUDA_SUCCESS;
 }
 
+// 4-D tiled map over the first `rows` rows of a [B, H, capacity, D] bf16
+// buffer (a KV cache): 64 x 128-row boxes, the same 128-byte-swizzled
+// shared-memory tile as make_bshd_map.  Rows at or past `rows` read as zero,
+// so a partly filled last tile never brings in stale cache contents.
+bool make_bhsd_map(CUtensorMap* map, const void* base, int B, int H, int rows, int capacity, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)capacity * D * 2, (cuuint64_t)H * capacity * D * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------- workspace maps
 struct PrefillWs {
   size_t lo, hi, table, q_hat, k_hat, total;
@@ -120,6 +137,41 @@ bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w) {
   off = align_up(off + rows * Hq * D * 2, 1024);
   w->k_hat = off;
   off = align_up(off + rows * Hkv * D * 2, 1024);
+  w->total = off;
+  return true;
+}
+
+// Chunked prefill: rows of history a local chunk reads from the ring.
+int chunk_hist(int start, g3_layer_kind kind, int window) {
+  return kind == G3_LAYER_LOCAL ? std::min(start, window - 1) : start;
+}
+struct ChunkWs {
+  size_t lo, hi, table, q_hat, ctx_k, ctx_v, total;
+  int rows;  // K/V rows of the local context buffers (history + chunk)
+};
+bool chunk_ws(int B, int C, int Hq, int Hkv, int D, int start, g3_layer_kind kind, int window, ChunkWs* w) {
+  if (B < 1 || C < 1 || Hq < 1 || Hkv < 1 || D < 1 || start < 0) return false;
+  if (kind == G3_LAYER_LOCAL && window < 1) return false;
+  const size_t rows = (size_t)B * C;
+  size_t off = g3::kHeaderBytes;
+  w->lo = off;
+  off = align_up(off + rows * 4, 1024);
+  w->hi = off;
+  off = align_up(off + rows * 4, 1024);
+  w->table = off;
+  off = align_up(off + rows * (D / 2) * 8, 1024);
+  w->q_hat = off;
+  off = align_up(off + rows * Hq * D * 2, 1024);
+  w->rows = 0;
+  w->ctx_k = w->ctx_v = off;
+  if (kind == G3_LAYER_LOCAL) {
+    w->rows = chunk_hist(start, kind, window) + C;
+    const size_t bytes = (size_t)B * Hkv * w->rows * D * 2;
+    w->ctx_k = off;
+    off = align_up(off + bytes, 1024);
+    w->ctx_v = off;
+    off = align_up(off + bytes, 1024);
+  }
   w->total = off;
   return true;
 }
@@ -169,6 +221,13 @@ const char* g3attn_last_error(void) { return g_last_error.c_str(); }
 size_t g3attn_prefill_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D) {
   PrefillWs w;
   if (!prefill_ws(B, S, Hq, Hkv, D, &w)) return 0;
+  return w.total;
+}
+
+size_t g3attn_prefill_chunk_workspace_size(int32_t B, int32_t C, int32_t Hq, int32_t Hkv, int32_t D, int32_t start,
+                                           g3_layer_kind layer_kind, int32_t window) {
+  ChunkWs w;
+  if (!chunk_ws(B, C, Hq, Hkv, D, start, layer_kind, window, &w)) return 0;
   return w.total;
 }
 
@@ -258,6 +317,7 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   pp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
   pp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
   pp.cache_cap = cache_capacity;
+  pp.total = S;
   pp.err = err;
 
   CUtensorMap tq, tk, tv;
@@ -286,6 +346,148 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill attention: %s", cudaGetErrorString(e));
+  return G3_OK;
+}
+
+g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, const float* q_gamma,
+                               const float* k_gamma, const int32_t* positions, void* k_cache, void* v_cache,
+                               int32_t cache_capacity, int32_t start, g3_layer_kind layer_kind, int32_t window,
+                               float rope_base, float interp_factor, const int32_t* image_spans, int32_t n_spans,
+                               int32_t B, int32_t C, int32_t Hq, int32_t Hkv, int32_t D, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !q_gamma || !k_gamma || !positions || !k_cache || !v_cache || !out)
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: a required pointer is NULL");
+  if (B < 1 || C < 1 || Hq < 1 || Hkv < 1 || D < 1 || start < 0)
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: sizes must be positive and start >= 0 (B=%d C=%d start=%d)", B, C,
+                start);
+  if (Hq % Hkv != 0) return fail(G3_ERR_INVALID_ARG, "prefill_chunk: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
+  if (layer_kind != G3_LAYER_LOCAL && layer_kind != G3_LAYER_GLOBAL)
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: bad layer kind %d", (int)layer_kind);
+  if (layer_kind == G3_LAYER_LOCAL && (window < 1 || cache_capacity != window))
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: local layers need window >= 1 and cache_capacity == window");
+  if (layer_kind == G3_LAYER_GLOBAL && (long long)cache_capacity < (long long)start + C)
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: global cache capacity %d < start + C = %lld", cache_capacity,
+                (long long)start + C);
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return fail(G3_ERR_INVALID_ARG, "prefill_chunk: bad rope_base");
+  if (!(interp_factor > 0.f) || !std::isfinite(interp_factor))
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: bad interp_factor");
+  if (n_spans < 0 || (n_spans > 0 && image_spans == nullptr) || (n_spans == 0 && image_spans != nullptr))
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: image_spans must be NULL iff n_spans == 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(k_cache) ||
+      !aligned16(v_cache))
+    return fail(G3_ERR_INVALID_ARG, "prefill_chunk: q, k, v, out and the caches must be 16-byte aligned");
+  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "prefill_chunk: head_dim %d not built (64, 128, 256)", D);
+  if ((long long)start + C > 0x7fffffffLL || (size_t)B * Hkv * cache_capacity * D >= (1ull << 40) ||
+      (size_t)B * C * Hq * D >= (1ull << 40))
+    return fail(G3_ERR_UNSUPPORTED, "prefill_chunk: problem too large");
+  const int G = Hq / Hkv;
+  const int hpc = (G % 2 == 0 && layer_kind == G3_LAYER_GLOBAL && D <= 128) ? 2 : 1;
+  const long long n_qtiles = (C + g3::kTileRows - 1) / g3::kTileRows;
+  if (n_qtiles * B * Hkv * (G / hpc) > 0x7fffffffLL) return fail(G3_ERR_UNSUPPORTED, "prefill_chunk: grid too large");
+
+  ChunkWs w;
+  chunk_ws(B, C, Hq, Hkv, D, start, layer_kind, window, &w);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(G3_ERR_WORKSPACE, "prefill_chunk: workspace NULL or not 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(G3_ERR_WORKSPACE, "prefill_chunk: workspace %zu bytes < required %zu", workspace_bytes, w.total);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* err = reinterpret_cast<int*>(ws);
+  const bool local = layer_kind == G3_LAYER_LOCAL;
+  // Keys the chunk can see, as rows of one [B, Hkv, rows, D] buffer: the cache
+  // itself on a global layer (token t in row t); on a local layer a context
+  // buffer holding the ring's last `hist` tokens and then the chunk.
+  const int hist = chunk_hist(start, layer_kind, window);
+  const int key_base = local ? start - hist : 0;
+  __nv_bfloat16* keys = local ? reinterpret_cast<__nv_bfloat16*>(ws + w.ctx_k) : static_cast<__nv_bfloat16*>(k_cache);
+  __nv_bfloat16* vals = local ? reinterpret_cast<__nv_bfloat16*>(ws + w.ctx_v) : static_cast<__nv_bfloat16*>(v_cache);
+  const int rows = local ? w.rows : cache_capacity;  // row capacity of `keys` / `vals`
+  const int visible = local ? hist + C : start + C;  // rows holding keys of tokens < start + C
+
+  g3::PrologueParams pp{};
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.q_gamma = q_gamma;
+  pp.k_gamma = k_gamma;
+  pp.positions = positions;
+  pp.spans = image_spans;
+  pp.n_spans = n_spans;
+  pp.B = B;
+  pp.S = C;
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.kind = (int)layer_kind;
+  pp.window = local ? window : start + C;
+  pp.rope_base = rope_base;
+  pp.interp = interp_factor;
+  for (int f = 0; f < D / 2; ++f) pp.inv_freq[f] = std::pow((double)rope_base, -2.0 * f / D);
+  pp.q_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.q_hat);
+  pp.k_hat = nullptr;  // keys go straight to their rows in `keys`
+  pp.lo = reinterpret_cast<int32_t*>(ws + w.lo);
+  pp.hi = reinterpret_cast<int32_t*>(ws + w.hi);
+  pp.rope_table = reinterpret_cast<float2*>(ws + w.table);
+  pp.k_cache = keys;
+  pp.v_cache = vals;
+  pp.cache_cap = rows;
+  pp.start = start;
+  pp.key_base = key_base;
+  pp.total = start + C;
+  pp.fill_rows = 1;
+  pp.err = err;
+
+  g3::RingCopyParams rp{};
+  rp.ring_k = static_cast<__nv_bfloat16*>(k_cache);
+  rp.ring_v = static_cast<__nv_bfloat16*>(v_cache);
+  rp.ctx_k = keys;
+  rp.ctx_v = vals;
+  rp.B = B;
+  rp.Hkv = Hkv;
+  rp.W = local ? window : 1;
+  rp.rows = rows;
+  rp.hist = hist;
+  rp.key_base = key_base;
+  rp.start = start;
+  rp.C = C;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_bshd_map(&tq, pp.q_hat, B, C, Hq, D) || !make_bhsd_map(&tk, keys, B, Hkv, visible, rows, D) ||
+      !make_bhsd_map(&tv, vals, B, Hkv, visible, rows, D))
+    return fail(G3_ERR_CUDA, "prefill_chunk: cuTensorMapEncodeTiled unavailable or failed");
+
+  cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk: %s", cudaGetErrorString(e));
+  if (local && hist > 0) {
+    e = traced("prefill_ring_gather", st, [&] { return g3::launch_ring_gather(rp, D, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk gather: %s", cudaGetErrorString(e));
+  }
+  e = traced("prefill_prologue", st, [&] { return g3::launch_prefill_prologue(pp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk prologue: %s", cudaGetErrorString(e));
+
+  g3::AttnParams ap{};
+  ap.lo = pp.lo;
+  ap.hi = pp.hi;
+  ap.kv_head_major = 1;
+  ap.out = static_cast<__nv_bfloat16*>(out);
+  ap.lse = lse;
+  ap.err = err;
+  ap.B = B;
+  ap.S = C;
+  ap.Hq = Hq;
+  ap.Hkv = Hkv;
+  ap.G = G;
+  ap.n_qtiles = (int)n_qtiles;
+  ap.n_groups = G / hpc;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk attention: %s", cudaGetErrorString(e));
+  if (local) {
+    e = traced("prefill_ring_write_back", st, [&] { return g3::launch_ring_write_back(rp, D, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk write-back: %s", cudaGetErrorString(e));
+  }
   return G3_OK;
 }
 

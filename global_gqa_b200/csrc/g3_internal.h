@@ -38,12 +38,18 @@ struct PrologueParams {
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   int cache_cap;
+  // Chunked prefill: this call's tokens are start .. start+S-1 of a sequence
+  // of `total` tokens; lo/hi count keys from token key_base; with fill_rows
+  // every token's key and value go to row start + t - key_base of k_cache /
+  // v_cache.  A whole prefill has start = key_base = 0, total = S, fill_rows 0.
+  int start, key_base, total, fill_rows;
   int* err;
 };
 
 struct AttnParams {
   const int32_t* lo;
   const int32_t* hi;
+  int kv_head_major;   // K/V tensor maps over [B, Hkv, rows, D] (a cache) instead of [B, S, Hkv, D]
   __nv_bfloat16* out;  // [B,S,Hq,D]
   float* lse;          // [B,Hq,S] or null
   int* err;
@@ -82,6 +88,19 @@ struct DecodeParams {
 // Launchers return the launch status; `name` receives a static kernel name
 // for tracing.
 cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st);
+// Chunked prefill on a local layer: copy the ring's history rows (tokens
+// key_base .. key_base+hist-1, slot t % W) to rows 0..hist-1 of the [B, Hkv,
+// rows, D] buffers ctx_k / ctx_v, or (write_back) the chunk's last min(C, W)
+// tokens from rows hist + j back into the ring.
+struct RingCopyParams {
+  __nv_bfloat16* ring_k;
+  __nv_bfloat16* ring_v;
+  __nv_bfloat16* ctx_k;
+  __nv_bfloat16* ctx_v;
+  int B, Hkv, W, rows, hist, key_base, start, C;
+};
+cudaError_t launch_ring_gather(const RingCopyParams& p, int D, cudaStream_t st);
+cudaError_t launch_ring_write_back(const RingCopyParams& p, int D, cudaStream_t st);
 cudaError_t launch_prefill_attention(const AttnParams& p, int D, int heads_per_cta, const CUtensorMap& tm_q,
                                      const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
 size_t prefill_attention_smem_bytes(int D, int heads_per_cta);

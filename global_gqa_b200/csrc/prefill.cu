@@ -143,17 +143,18 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
         const int s = t % NS;
         const uint32_t ph = (t / NS) & 1;
         const int kv0 = (t_begin + t) * 128;
+        // Tile coordinates: [B, S, Hkv, D] maps take (head, row); [B, Hkv,
+        // rows, D] maps over a cache take (row, head).
+        const int c1 = p.kv_head_major ? kv0 : kvh, c2 = p.kv_head_major ? kvh : kv0;
         if (!mbar_wait(&bars->k_empty[s], ph ^ 1, abort, p.err, 1)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], L::kTile);
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(smem + L::kK + s * L::kTile + kb * kSwizzleBlock, &tm_k, &bars->k_full[s], kb * 64, kvh,
-                      kv0, b);
+          tma_load_4d(smem + L::kK + s * L::kTile + kb * kSwizzleBlock, &tm_k, &bars->k_full[s], kb * 64, c1, c2, b);
         last_k[s] = ph;
         if (!mbar_wait(&bars->v_empty[s], ph ^ 1, abort, p.err, 2)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], L::kTile);
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(smem + L::kV + s * L::kTile + kb * kSwizzleBlock, &tm_v, &bars->v_full[s], kb * 64, kvh,
-                      kv0, b);
+          tma_load_4d(smem + L::kV + s * L::kTile + kb * kSwizzleBlock, &tm_v, &bars->v_full[s], kb * 64, c1, c2, b);
         last_v[s] = ph;
       }
       // Let every copy this thread started land before the block can exit.

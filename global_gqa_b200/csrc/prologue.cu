@@ -28,6 +28,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <algorithm>
 #include <cstdint>
 
 #include "g3_internal.h"
@@ -57,25 +58,30 @@ __global__ void __launch_bounds__(kTableThreads) rope_table_kernel(PrologueParam
   p.rope_table[idx] = make_float2((float)cd, (float)sd);
 
   if (f == 0) {
-    int lo = (p.kind == 1) ? 0 : max(0, t - p.window + 1);
-    int hi = t;
+    // Interval of token ta (whole-sequence index), as key rows from key_base.
+    const int ta = p.start + t;
+    int lo = (p.kind == 1) ? 0 : max(0, ta - p.window + 1);
+    int hi = ta;
     const int32_t* sp = p.spans + (size_t)b * p.n_spans * 2;
     for (int k = 0; k < p.n_spans; ++k) {
       const int st = sp[2 * k], en = sp[2 * k + 1];
-      if (st <= t && t < en) {
+      if (st <= ta && ta < en) {
         lo = min(lo, max(st, 0));
-        hi = max(hi, min(en, p.S) - 1);
+        hi = max(hi, min(en, p.total) - 1);
         break;
       }
     }
-    p.lo[bt] = lo;
-    p.hi[bt] = hi;
+    p.lo[bt] = lo - p.key_base;
+    p.hi[bt] = hi - p.key_base;
     if (t == 0 && p.n_spans > 0) {
+      // Sorted, disjoint, inside the sequence, and (chunked prefill) not
+      // holding tokens on both sides of the chunk's first or last boundary.
       int prev_end = 0;
       bool ok = true;
       for (int k = 0; k < p.n_spans; ++k) {
         const int st = sp[2 * k], en = sp[2 * k + 1];
-        ok = ok && st >= prev_end && st < en && en <= p.S;
+        ok = ok && st >= prev_end && st < en && en <= p.total;
+        ok = ok && !(st < p.start && en > p.start) && !(st < p.total && en > p.total);
         prev_end = en;
       }
       if (!ok) record_error(p.err, kErrInvalid, 100);
@@ -177,14 +183,17 @@ __global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(ProloguePa
         } else {
           const int kh = h - p.Hq;
           const size_t row = (size_t)bt * p.Hkv + kh;
-          __nv_bfloat16* dst = p.k_hat + row * D;
-          *reinterpret_cast<uint4*>(dst + d1) = lo8;
-          *reinterpret_cast<uint4*>(dst + H2 + d1) = hi8;
+          if (p.k_hat != nullptr) {
+            __nv_bfloat16* dst = p.k_hat + row * D;
+            *reinterpret_cast<uint4*>(dst + d1) = lo8;
+            *reinterpret_cast<uint4*>(dst + H2 + d1) = hi8;
+          }
           if (p.k_cache != nullptr) {
             const int b = bt / p.S, t = bt % p.S;
-            const bool write = (p.kind == 1) ? (t < p.cache_cap) : (t >= p.S - p.cache_cap);
+            const bool write =
+                p.fill_rows || ((p.kind == 1) ? (t < p.cache_cap) : (t >= p.S - p.cache_cap));
             if (write) {
-              const int slot = (p.kind == 1) ? t : t % p.cache_cap;
+              const int slot = p.fill_rows ? p.start + t - p.key_base : (p.kind == 1) ? t : t % p.cache_cap;
               const size_t crow = ((size_t)b * p.Hkv + kh) * p.cache_cap + slot;
               *reinterpret_cast<uint4*>(p.k_cache + crow * D + d1) = lo8;
               *reinterpret_cast<uint4*>(p.k_cache + crow * D + H2 + d1) = hi8;
@@ -219,6 +228,61 @@ cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t
     return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+// ======================================================= ring copies (local chunks)
+// One thread per 16 bytes of a row; rows are (sequence, kv head, token).
+constexpr int kRingThreads = 256;
+
+template <int D, bool WRITE_BACK>
+__global__ void __launch_bounds__(kRingThreads) ring_copy_kernel(RingCopyParams p) {
+  constexpr int V16 = D / 8;  // 16-byte pieces per row
+  const int n_tok = WRITE_BACK ? min(p.C, p.W) : p.hist;
+  const size_t total = (size_t)p.B * p.Hkv * n_tok * V16;
+  for (size_t i = (size_t)blockIdx.x * kRingThreads + threadIdx.x; i < total; i += (size_t)gridDim.x * kRingThreads) {
+    const int v = (int)(i % V16);
+    const size_t r = i / V16;
+    const int j = (int)(r % n_tok);
+    const size_t bh = r / n_tok;  // b * Hkv + kv head
+    // Token of this row (whole-sequence index) and its ring slot / buffer row.
+    const int tok = WRITE_BACK ? p.start + (p.C - n_tok) + j : p.key_base + j;
+    const int ctx_row = tok - p.key_base;
+    const size_t ring = (bh * p.W + (tok % p.W)) * V16 + v;
+    const size_t ctx = (bh * p.rows + ctx_row) * V16 + v;
+    uint4* rk = reinterpret_cast<uint4*>(p.ring_k);
+    uint4* rv = reinterpret_cast<uint4*>(p.ring_v);
+    uint4* ck = reinterpret_cast<uint4*>(p.ctx_k);
+    uint4* cv = reinterpret_cast<uint4*>(p.ctx_v);
+    if (WRITE_BACK) {
+      rk[ring] = ck[ctx];
+      rv[ring] = cv[ctx];
+    } else {
+      ck[ctx] = rk[ring];
+      cv[ctx] = rv[ring];
+    }
+  }
+}
+
+template <bool WB>
+static cudaError_t launch_ring_t(const RingCopyParams& p, int D, cudaStream_t st) {
+  const long long n_tok = WB ? std::min(p.C, p.W) : p.hist;
+  const long long work = (long long)p.B * p.Hkv * n_tok * (D / 8);
+  if (work == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)std::min<long long>((work + kRingThreads - 1) / kRingThreads, 148 * 16);
+  if (D == 128)
+    ring_copy_kernel<128, WB><<<blocks, kRingThreads, 0, st>>>(p);
+  else if (D == 64)
+    ring_copy_kernel<64, WB><<<blocks, kRingThreads, 0, st>>>(p);
+  else if (D == 256)
+    ring_copy_kernel<256, WB><<<blocks, kRingThreads, 0, st>>>(p);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_gather(const RingCopyParams& p, int D, cudaStream_t st) { return launch_ring_t<false>(p, D, st); }
+cudaError_t launch_ring_write_back(const RingCopyParams& p, int D, cudaStream_t st) {
+  return launch_ring_t<true>(p, D, st);
 }
 
 }  // namespace g3

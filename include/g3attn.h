@@ -103,6 +103,53 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v,
                          void* k_cache, void* v_cache, int32_t cache_capacity,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------- chunked prefill
+ * Bytes of workspace g3attn_prefill_chunk needs for these sizes (0 if the
+ * sizes are invalid).  The workspace must be 256-byte aligned.
+ */
+size_t g3attn_prefill_chunk_workspace_size(int32_t B, int32_t C, int32_t Hq, int32_t Hkv, int32_t D,
+                                           int32_t start, g3_layer_kind layer_kind, int32_t window);
+
+/*
+ * Chunked prefill: the next C tokens of B sequences whose first `start`
+ * tokens are already in the KV cache.  The result equals rows start ..
+ * start+C-1 of g3attn_prefill over all start + C tokens: the same local or
+ * global mask of Gemma 3 (Technical Report, sections 1 and 2), with a long
+ * prompt taken in pieces.
+ *
+ *   q, k, v    bf16 [B, C, Hq|Hkv, D]  raw projections of the chunk's tokens
+ *   q_gamma, k_gamma, layer_kind, window, rope_base, interp_factor
+ *              as for g3attn_prefill
+ *   positions  int32 [B, C]  RoPE positions of the chunk's tokens
+ *   k_cache, v_cache bf16 [B, Hkv, cache_capacity, D], required: rotated keys
+ *              and values of tokens 0 .. start-1 as g3attn_prefill (with
+ *              caches) or earlier chunks left them.  GLOBAL: token t in slot t,
+ *              cache_capacity >= start + C.  LOCAL: a ring of cache_capacity ==
+ *              window slots, token t in slot t % window, holding the last
+ *              min(start, window) tokens.  The chunk's tokens are added the
+ *              same way (the call reads the ring before it overwrites it).
+ *   start      >= 0: tokens already cached; the same for every sequence
+ *   image_spans int32 [B, n_spans, 2] half-open, in token indices of the whole
+ *              sequence, sorted, disjoint, end <= start + C; no span may hold
+ *              tokens on both sides of `start` or of start + C (an image never
+ *              crosses a chunk boundary).  NULL iff n_spans == 0.  A violation
+ *              found on the device is reported by g3attn_check_device_error().
+ *   B, C, Hq, Hkv, D   C >= 1; as for g3attn_prefill otherwise
+ *   out        bf16 [B, C, Hq, D];  lse optional fp32 [B, Hq, C]
+ *   workspace  >= g3attn_prefill_chunk_workspace_size(...) bytes
+ */
+g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v,
+                               const float* q_gamma, const float* k_gamma,
+                               const int32_t* positions,
+                               void* k_cache, void* v_cache, int32_t cache_capacity,
+                               int32_t start,
+                               g3_layer_kind layer_kind, int32_t window,
+                               float rope_base, float interp_factor,
+                               const int32_t* image_spans, int32_t n_spans,
+                               int32_t B, int32_t C, int32_t Hq, int32_t Hkv, int32_t D,
+                               void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------- decode
  * Bytes of workspace g3attn_decode needs (0 if the sizes are invalid).
  */
