@@ -275,6 +275,75 @@ def run_gpu(args, rank, world, local_rank):
             "flops": f, "attention_us": 1e3 * ma / na, "attention_tflops": f / (ma / na * 1e-3) / 1e12,
             "prologue_us": 1e3 * mpro / npro}
 
+    # ---- chunked prefill (outside the timed region): the same block, each layer's
+    # 8192-token prompt taken as four 2048-token chunks onto its KV cache
+    chunked = None
+    if args.extras:
+        C = 2048
+        cws = None
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        caches = []
+        for L, x in layers:
+            cap = L.window if L.kind == 0 else cfg.S
+            caches.append((torch.empty(cfg.B, cfg.Hkv, cap, cfg.D, dtype=torch.bfloat16, device=dev),
+                           torch.empty(cfg.B, cfg.Hkv, cap, cfg.D, dtype=torch.bfloat16, device=dev)))
+        need = max(g3.prefill_chunk_workspace_size(cfg.B, C, cfg.Hq, cfg.Hkv, cfg.D, a, L.kind, L.window)
+                   for L, _ in layers for a in range(0, cfg.S, C))
+        cws = torch.empty(need, dtype=torch.uint8, device=dev)
+        pieces = [[{k: x[k][:, a:a + C].contiguous() for k in ("q", "k", "v", "positions")}
+                   for a in range(0, cfg.S, C)] for _, x in layers]
+
+        def chunked_block():
+            for (L, x), (kc, vc), ps in zip(layers, caches, pieces):
+                for i, pc in enumerate(ps):
+                    g3.prefill_chunk(pc["q"], pc["k"], pc["v"], x["q_gamma"], x["k_gamma"], pc["positions"], kc, vc,
+                                     i * C, L.kind, L.window, L.rope_base, L.interp, None, ws=cws, stream=stream)
+
+        for _ in range(2):
+            chunked_block()
+        barrier()
+        reps = max(args.steps // 2, 3)
+        ev0.record(stream)
+        for _ in range(reps):
+            chunked_block()
+        ev1.record(stream)
+        barrier()
+        cms = ev0.elapsed_time(ev1) / reps
+        chunked = {"workload": f"{cfg.name} as {cfg.S // C} chunks of {C} tokens per layer (no image spans)",
+                   "ms_per_block": cms, "tflops": block_flops / (cms * 1e-3) / 1e12}
+        del caches, cws, pieces
+
+    # ---- Gemma 3 1B attention shapes (outside the timed region): one local and
+    # one global layer of 32768 tokens, 4 query heads, 1 kv head, head dim 256
+    shapes_1b = None
+    if args.extras:
+        S1, Hq1, Hkv1, D1 = 32768, 4, 1, 256
+        x1 = {k: v.to(dev) for k, v in inputs.prefill_layer_inputs(1, S1, Hq1, Hkv1, D1, seed=0, layer=0).items()
+              if v is not None}
+        out1 = torch.empty_like(x1["q"])
+        ws1 = torch.empty(g3.prefill_workspace_size(1, S1, Hq1, Hkv1, D1), dtype=torch.uint8, device=dev)
+        shapes_1b = {"workload": "B1 S32768 Hq4 Hkv1 D256 (Gemma 3 1B shapes)"}
+        for kind, W, base, interp, name in ((0, 1024, 1e4, 1.0, "local"), (1, S1, 1e6, 8.0, "global")):
+            f = metrics.layer_flops(1, S1, Hq1, D1, kind, W)
+            for _ in range(2):
+                g3.prefill(x1["q"], x1["k"], x1["v"], x1["q_gamma"], x1["k_gamma"], x1["positions"], kind, W, base,
+                           interp, out=out1, ws=ws1, stream=stream)
+            g3.trace_collect()
+            barrier()
+            g3.trace_enable(True)
+            for _ in range(5):
+                g3.prefill(x1["q"], x1["k"], x1["v"], x1["q_gamma"], x1["k_gamma"], x1["positions"], kind, W, base,
+                           interp, out=out1, ws=ws1, stream=stream)
+            barrier()
+            g3.trace_enable(False)
+            tr = g3.trace_collect()
+            na, ma = tr.get("prefill_attention", (1, 0.0))
+            npro, mpro = tr.get("prefill_prologue", (1, 0.0))
+            shapes_1b[name] = {"flops": f, "attention_us": 1e3 * ma / na,
+                               "attention_tflops": f / (ma / na * 1e-3) / 1e12, "prologue_us": 1e3 * mpro / npro}
+        del x1, out1, ws1
+
     # ---- end to end through the public API from pinned host memory
     host = []
     for L, x in layers:
@@ -324,6 +393,8 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": roofline,
         "kernels": kernels,
         "layer_kinds": layer_kinds,
+        "chunked_prefill": chunked,
+        "shapes_1b": shapes_1b,
         "gpu_launches": sum(v[0] for v in trace.values()),
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -428,6 +499,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="g3attn", choices=["g3attn", "reference"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the chunked-prefill and 1B-shape measurements")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
