@@ -22,3 +22,4 @@ from .attention import (  # noqa: F401
     decode,
     unmasked_pairs,
 )
+from .projector import soft_tokens  # noqa: F401,E402
