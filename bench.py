@@ -344,6 +344,33 @@ def run_gpu(args, rank, world, local_rank):
                                "attention_tflops": f / (ma / na * 1e-3) / 1e12, "prologue_us": 1e3 * mpro / npro}
         del x1, out1, ws1
 
+    # ---- image soft tokens (outside the timed region): 64 images, 64x64 patch
+    # grid of 1152 features each, 4x4 pool -> 256 tokens; HBM-bound
+    soft = None
+    if args.extras:
+        Bi, gh, F = 64, 64, 1152
+        px = torch.empty(Bi, gh * gh, F, dtype=torch.bfloat16, device=dev)
+        inputs.device_fill_normal_bf16(px, seed=17)
+        gam = torch.ones(F, dtype=torch.float32, device=dev)
+        so = torch.empty(Bi, (gh // 4) ** 2, F, dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            g3.soft_tokens(px, gam, gh, gh, 4, out=so, stream=stream)
+        e0s = torch.cuda.Event(enable_timing=True)
+        e1s = torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0s.record(stream)
+        for _ in range(20):
+            g3.soft_tokens(px, gam, gh, gh, 4, out=so, stream=stream)
+        e1s.record(stream)
+        barrier()
+        sms = e0s.elapsed_time(e1s) / 20
+        sbytes = (px.numel() + so.numel()) * 2 + F * 4
+        gbs = sbytes / (sms * 1e-3) / 1e9
+        soft = {"workload": "64 images, 64x64 patches x 1152 features, 4x4 pool -> 256 tokens",
+                "us": sms * 1e3, "bytes": sbytes, "GB/s": gbs, "frac_of_measured_hbm": gbs / pk["hbm_gbs"],
+                "note": "inputs 604 MB > L2, re-read each call"}
+        del px, so
+
     # ---- end to end through the public API from pinned host memory
     host = []
     for L, x in layers:
@@ -395,6 +422,7 @@ def run_gpu(args, rank, world, local_rank):
         "layer_kinds": layer_kinds,
         "chunked_prefill": chunked,
         "shapes_1b": shapes_1b,
+        "soft_tokens": soft,
         "gpu_launches": sum(v[0] for v in trace.values()),
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -46,6 +46,7 @@ _SIGS = {
     "g3attn_prefill_chunk": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_int, _i32,
                                             _f32, _f32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
                                             _sz, _vp]),
+    "g3attn_soft_tokens": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "g3attn_decode_workspace_size": (_sz, [_i32] * 5),
     "g3attn_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, ctypes.c_int, _i32,
                                      _f32, _f32, _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
@@ -283,3 +284,24 @@ def prefill_chunk(q, k, v, q_gamma, k_gamma, positions, k_cache, v_cache, start:
                                     _stream_ptr(stream, q.device))
     _check(st, "g3attn_prefill_chunk")
     return (out, lse) if return_lse else out
+
+
+def soft_tokens(patches, gamma, grid_h: int, grid_w: int, pool: int = 4, *, out=None, stream=None):
+    """Image soft tokens: pool x pool average of the patch grid, then RMS norm times gamma.
+
+    patches bf16 [B, grid_h*grid_w, F], gamma fp32 [F]; returns bf16 [B, (grid_h/pool)*(grid_w/pool), F].
+    """
+    torch = _torch()
+    _req(patches, "patches", torch.bfloat16)
+    if patches.dim() != 3 or patches.shape[1] != grid_h * grid_w:
+        raise ValueError("patches must be [B, grid_h * grid_w, F]")
+    B, _, F = patches.shape
+    _req(gamma, "gamma", torch.float32, (F,))
+    n_out = (grid_h // pool) * (grid_w // pool)
+    if out is None:
+        out = torch.empty(B, n_out, F, dtype=torch.bfloat16, device=patches.device)
+    _req(out, "out", torch.bfloat16, (B, n_out, F))
+    st = lib().g3attn_soft_tokens(_ptr(patches), _ptr(gamma), B, grid_h, grid_w, F, pool, _ptr(out),
+                                  _stream_ptr(stream, patches.device))
+    _check(st, "g3attn_soft_tokens")
+    return out

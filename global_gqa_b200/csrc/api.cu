@@ -569,6 +569,38 @@ g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new, con
   return G3_OK;
 }
 
+g3_status g3attn_soft_tokens(const void* patches, const float* gamma, int32_t B, int32_t grid_h, int32_t grid_w,
+                             int32_t F, int32_t pool, void* out, void* stream) {
+  g_last_error.clear();
+  if (!patches || !gamma || !out) return fail(G3_ERR_INVALID_ARG, "soft_tokens: a required pointer is NULL");
+  if (B < 1 || grid_h < 1 || grid_w < 1 || F < 8 || pool < 1)
+    return fail(G3_ERR_INVALID_ARG, "soft_tokens: sizes must be positive (B=%d grid %dx%d F=%d pool=%d)", B, grid_h,
+                grid_w, F, pool);
+  if (grid_h % pool != 0 || grid_w % pool != 0)
+    return fail(G3_ERR_INVALID_ARG, "soft_tokens: grid %dx%d is not a multiple of pool %d", grid_h, grid_w, pool);
+  if (!aligned16(patches) || !aligned16(gamma) || !aligned16(out))
+    return fail(G3_ERR_INVALID_ARG, "soft_tokens: patches, gamma and out must be 16-byte aligned");
+  if (F % 8 != 0 || F > 8 * g3::kSoftTokenMaxThreads)
+    return fail(G3_ERR_UNSUPPORTED, "soft_tokens: F=%d not built (a multiple of 8 up to %d)", F,
+                8 * g3::kSoftTokenMaxThreads);
+  if (pool != 1 && pool != 2 && pool != 4) return fail(G3_ERR_UNSUPPORTED, "soft_tokens: pool %d not built (1, 2, 4)", pool);
+  if ((long long)B * (grid_h / pool) * (grid_w / pool) > 0x7fffffffLL || (size_t)B * grid_h * grid_w * F >= (1ull << 40))
+    return fail(G3_ERR_UNSUPPORTED, "soft_tokens: problem too large");
+  g3::SoftTokenParams sp{};
+  sp.patches = static_cast<const __nv_bfloat16*>(patches);
+  sp.gamma = gamma;
+  sp.out = static_cast<__nv_bfloat16*>(out);
+  sp.B = B;
+  sp.grid_h = grid_h;
+  sp.grid_w = grid_w;
+  sp.F = F;
+  sp.pool = pool;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = traced("soft_tokens", st, [&] { return g3::launch_soft_tokens(sp, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "soft_tokens: %s", cudaGetErrorString(e));
+  return G3_OK;
+}
+
 g3_status g3attn_check_device_error(void* workspace, void* stream) {
   if (workspace == nullptr) return fail(G3_ERR_WORKSPACE, "check: workspace is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -108,6 +108,17 @@ size_t prefill_attention_smem_bytes(int D, int heads_per_cta);
 // Sets the calling thread's g3attn_last_error() text.
 void set_last_error(const char* msg);
 
+// Image soft tokens: pool x pool average of a grid_h x grid_w patch grid, then
+// RMS norm over F features times gamma.
+constexpr int kSoftTokenMaxThreads = 1024;
+struct SoftTokenParams {
+  const __nv_bfloat16* patches;  // [B, grid_h * grid_w, F]
+  const float* gamma;            // [F]
+  __nv_bfloat16* out;            // [B, (grid_h / pool) * (grid_w / pool), F]
+  int B, grid_h, grid_w, F, pool;
+};
+cudaError_t launch_soft_tokens(const SoftTokenParams& p, cudaStream_t st);
+
 cudaError_t launch_decode_prologue(const DecodeParams& p, int D, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeParams& p, int D, int grid_chunks, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeParams& p, int D, cudaStream_t st);

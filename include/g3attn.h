@@ -150,6 +150,25 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v,
                                void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* -------------------------------------------------------------- soft tokens
+ * Image soft tokens of the multimodal projector ("Gemma explained: what's new
+ * in Gemma 3", 27B printout: RMSNorm over the vision features with eps 1e-6,
+ * and a 4x4 average pool with stride 4).  Each pool x pool block of an image's
+ * patch grid (raster order) is averaged, then RMS-normalised over its F
+ * features and multiplied by gamma.  An 896x896 image in 14x14 patches is a
+ * 64x64 grid, i.e. 256 soft tokens.  The projection to the language model's
+ * width (a trained matrix) is not part of this call.
+ *
+ *   patches   bf16 [B, grid_h * grid_w, F]   vision features, 16-byte aligned
+ *   gamma     fp32 [F]                       gain (multiplier), 16-byte aligned
+ *   grid_h, grid_w, pool   pool in {1, 2, 4}; grid_h and grid_w multiples of pool
+ *   F         multiple of 8, 8 <= F <= 8192
+ *   out       bf16 [B, (grid_h/pool) * (grid_w/pool), F], 16-byte aligned
+ * No workspace; asynchronous on `stream`.
+ */
+g3_status g3attn_soft_tokens(const void* patches, const float* gamma, int32_t B, int32_t grid_h,
+                             int32_t grid_w, int32_t F, int32_t pool, void* out, void* stream);
+
 /* ------------------------------------------------------------------- decode
  * Bytes of workspace g3attn_decode needs (0 if the sizes are invalid).
  */

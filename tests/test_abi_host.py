@@ -92,6 +92,52 @@ def test_decode_rejects_on_host(lib, kw, code):
     assert _decode(lib, **kw) == code
 
 
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, qg=FAKE, kg=FAKE, pos=FAKE, kc=FAKE, vc=FAKE, cap=1024, start=100, kind=0,
+             window=1024, base=1e4, interp=1.0, spans=None, n_spans=0, B=1, C=128, Hq=4, Hkv=2, D=128, out=FAKE,
+             lse=None, ws=FAKE * 256, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.g3attn_prefill_chunk(a["q"], a["k"], a["v"], a["qg"], a["kg"], a["pos"], a["kc"], a["vc"], a["cap"],
+                                    a["start"], a["kind"], a["window"], a["base"], a["interp"], a["spans"],
+                                    a["n_spans"], a["B"], a["C"], a["Hq"], a["Hkv"], a["D"], a["out"], a["lse"],
+                                    a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kc=None), 1), (dict(start=-1), 1), (dict(C=0), 1), (dict(cap=512), 1),
+    (dict(kind=1, cap=200), 1), (dict(Hq=3), 1), (dict(vc=FAKE + 8), 1), (dict(n_spans=1), 1),
+    (dict(D=96), 2), (dict(ws=None), 3), (dict(wsb=1000), 3),
+])
+def test_prefill_chunk_rejects_on_host(lib, kw, code):
+    assert _chunk(lib, **kw) == code
+    assert lib.g3attn_last_error() != b""
+
+
+def test_prefill_chunk_workspace_sizes(lib):
+    assert lib.g3attn_prefill_chunk_workspace_size(1, 0, 4, 2, 128, 0, 0, 1024) == 0
+    assert lib.g3attn_prefill_chunk_workspace_size(1, 16, 4, 2, 128, -1, 0, 1024) == 0
+    loc = lib.g3attn_prefill_chunk_workspace_size(1, 2048, 32, 16, 128, 6144, 0, 1024)
+    glb = lib.g3attn_prefill_chunk_workspace_size(1, 2048, 32, 16, 128, 6144, 1, 1024)
+    # a local chunk also holds its context: 1023 ring rows + the chunk, K and V
+    assert loc >= glb + 2 * 16 * (1023 + 2048) * 128 * 2
+    assert glb >= 2048 * 32 * 128 * 2 and glb % 1024 == 0
+
+
+def _soft(lib, **kw):
+    a = dict(p=FAKE, g=FAKE, B=2, gh=64, gw=64, F=1152, pool=4, out=FAKE, stream=None)
+    a.update(kw)
+    return lib.g3attn_soft_tokens(a["p"], a["g"], a["B"], a["gh"], a["gw"], a["F"], a["pool"], a["out"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(p=None), 1), (dict(out=None), 1), (dict(B=0), 1), (dict(F=4), 1), (dict(gh=62), 1),
+    (dict(g=FAKE + 4), 1), (dict(F=12), 2), (dict(F=8200), 2), (dict(pool=3, gh=63, gw=63), 2),
+])
+def test_soft_tokens_rejects_on_host(lib, kw, code):
+    assert _soft(lib, **kw) == code
+    assert lib.g3attn_last_error() != b""
+
+
 def test_check_device_error_null(lib):
     assert lib.g3attn_check_device_error(None, None) == 3
 
