@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
   const int hi_first = p.hi[rowbase + r0];     // smallest hi of the tile's rows
   const int t_begin = lo_first / 128;
   const int n_tiles = max(hi_last / 128, t_begin) - t_begin + 1;
+  const int n_pre = min(n_tiles, NS);  // K/V tiles loaded before the CTA-wide barrier
 
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
@@ -118,6 +119,26 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
+    // Thread 0 is also the TMA producer: start the Q tiles and the first K/V
+    // stages now, so their latency overlaps the TMEM allocation and the
+    // CTA-wide barrier below (the ring's empty barriers start released).
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    mbar_arrive_expect_tx(&bars->q_full, HPC * L::kTile);
+    for (int h = 0; h < HPC; ++h)
+      for (int kb = 0; kb < KB; ++kb)
+        tma_load_4d(smem + L::kQ + h * L::kTile + kb * kSwizzleBlock, &tm_q, &bars->q_full, kb * 64, h0 + h, r0, b);
+    for (int t = 0; t < n_pre; ++t) {
+      const int kv0 = (t_begin + t) * 128;
+      const int c1 = p.kv_head_major ? kv0 : kvh, c2 = p.kv_head_major ? kvh : kv0;
+      mbar_arrive_expect_tx(&bars->k_full[t], L::kTile);
+      for (int kb = 0; kb < KB; ++kb)
+        tma_load_4d(smem + L::kK + t * L::kTile + kb * kSwizzleBlock, &tm_k, &bars->k_full[t], kb * 64, c1, c2, b);
+      mbar_arrive_expect_tx(&bars->v_full[t], L::kTile);
+      for (int kb = 0; kb < KB; ++kb)
+        tma_load_4d(smem + L::kV + t * L::kTile + kb * kSwizzleBlock, &tm_v, &bars->v_full[t], kb * 64, c1, c2, b);
+    }
   }
   if (warp == 1) tmem_alloc(&bars->tmem_base, L::kTmemCols);
   tc_fence_before();
@@ -130,16 +151,10 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
    if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
+      // Tiles 0 .. n_pre-1 were started before the CTA-wide barrier.
       int last_k[3] = {-1, -1, -1}, last_v[3] = {-1, -1, -1};
-      mbar_arrive_expect_tx(&bars->q_full, HPC * L::kTile);
-      for (int h = 0; h < HPC; ++h)
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(smem + L::kQ + h * L::kTile + kb * kSwizzleBlock, &tm_q, &bars->q_full, kb * 64, h0 + h,
-                      r0, b);
-      for (int t = 0; t < n_tiles; ++t) {
+      for (int t = 0; t < n_pre; ++t) last_k[t] = last_v[t] = 0;
+      for (int t = n_pre; t < n_tiles; ++t) {
         const int s = t % NS;
         const uint32_t ph = (t / NS) & 1;
         const int kv0 = (t_begin + t) * 128;
