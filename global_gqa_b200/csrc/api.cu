@@ -320,9 +320,10 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   pp.total = S;
   pp.err = err;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_bshd_map(&tq, pp.q_hat, B, S, Hq, D) || !make_bshd_map(&tk, pp.k_hat, B, S, Hkv, D) ||
-      !make_bshd_map(&tv, v, B, S, Hkv, D))
+      !make_bshd_map(&tv, v, B, S, Hkv, D) ||
+      !make_bshd_map(&to, out, B, S, Hq, D))
     return fail(G3_ERR_CUDA, "prefill: cuTensorMapEncodeTiled unavailable or failed");
 
   cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
@@ -344,7 +345,7 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, st); });
+  e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill attention: %s", cudaGetErrorString(e));
   return G3_OK;
 }
@@ -453,9 +454,10 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
   rp.start = start;
   rp.C = C;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_bshd_map(&tq, pp.q_hat, B, C, Hq, D) || !make_bhsd_map(&tk, keys, B, Hkv, visible, rows, D) ||
-      !make_bhsd_map(&tv, vals, B, Hkv, visible, rows, D))
+      !make_bhsd_map(&tv, vals, B, Hkv, visible, rows, D) ||
+      !make_bshd_map(&to, out, B, C, Hq, D))
     return fail(G3_ERR_CUDA, "prefill_chunk: cuTensorMapEncodeTiled unavailable or failed");
 
   cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
@@ -482,7 +484,7 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, st); });
+  e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk attention: %s", cudaGetErrorString(e));
   if (local) {
     e = traced("prefill_ring_write_back", st, [&] { return g3::launch_ring_write_back(rp, D, st); });

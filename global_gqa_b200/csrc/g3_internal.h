@@ -102,7 +102,8 @@ struct RingCopyParams {
 cudaError_t launch_ring_gather(const RingCopyParams& p, int D, cudaStream_t st);
 cudaError_t launch_ring_write_back(const RingCopyParams& p, int D, cudaStream_t st);
 cudaError_t launch_prefill_attention(const AttnParams& p, int D, int heads_per_cta, const CUtensorMap& tm_q,
-                                     const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
+                                     const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_out,
+                                     cudaStream_t st);
 size_t prefill_attention_smem_bytes(int D, int heads_per_cta);
 
 // Sets the calling thread's g3attn_last_error() text.

@@ -62,6 +62,7 @@ struct AttnBarriers {
   uint64_t q_full;
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t out_ready[2];  // a head's output tile is staged in shared memory
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -70,7 +71,8 @@ struct AttnBarriers {
 template <int D, int HPC>
 __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMinBlocks)
     prefill_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
+                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                             AttnParams p) {
   using L = AttnLayout<D, HPC>;
   constexpr int NS = L::kStages;
   constexpr int KB = D / 64;  // swizzle columns per tile
@@ -115,6 +117,7 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
       mbar_init(&bars->s_full[h], 1);
       mbar_init(&bars->p_full[h], 256);
       mbar_init(&bars->o_full[h], 1);
+      mbar_init(&bars->out_ready[h], 8);  // softmax warps of the head
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -373,8 +376,12 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
         tc_fence_after();
         const float inv_a = 1.f / l_a, inv_b = 1.f / l_b;
         const int hq = h0 + h;
-        __nv_bfloat16* da = p.out + ((rowbase + r0 + ra) * p.Hq + hq) * D + 2 * m4;
-        __nv_bfloat16* db = p.out + ((rowbase + r0 + rb) * p.Hq + hq) * D + 2 * m4;
+        // O / l in bf16 is staged in this head's Q tile (no MMA reads it any
+        // more: every MMA completed before o_full) in the 128-byte-swizzled
+        // layout of a TMA tile, then one thread stores the tile.  Rows past S
+        // are clipped by the store.
+        uint8_t* stage = smem + L::kQ + h * L::kTile;
+        const int sw = ra & 7;  // rb = ra + 8 has the same swizzle phase
 #pragma unroll
         for (int q = 0; q < D / 64; ++q) {
           float o[32];
@@ -382,10 +389,19 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const int c = q * 64 + 8 * k;
-            if (valid_a) *reinterpret_cast<uint32_t*>(da + c) = pack_bf16x2(o[4 * k] * inv_a, o[4 * k + 1] * inv_a);
-            if (valid_b)
-              *reinterpret_cast<uint32_t*>(db + c) = pack_bf16x2(o[4 * k + 2] * inv_b, o[4 * k + 3] * inv_b);
+            uint8_t* blk = stage + q * kSwizzleBlock + ((k ^ sw) * 16) + m4 * 4;
+            *reinterpret_cast<uint32_t*>(blk + ra * 128) = pack_bf16x2(o[4 * k] * inv_a, o[4 * k + 1] * inv_a);
+            *reinterpret_cast<uint32_t*>(blk + rb * 128) = pack_bf16x2(o[4 * k + 2] * inv_b, o[4 * k + 3] * inv_b);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->out_ready[h]);
+        if (((warp - SW0) & 7) == 0 && lane == 0) {
+          if (mbar_wait(&bars->out_ready[h], 0, abort, p.err, 22)) {
+            for (int kb = 0; kb < KB; ++kb) tma_store_4d(&tm_out, stage + kb * kSwizzleBlock, kb * 64, hq, r0, b);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging tile must outlive the store's reads
           }
         }
         if (m4 == 0 && p.lse != nullptr) {
@@ -414,7 +430,7 @@ size_t prefill_attention_smem_bytes(int D, int hpc) {
 
 template <int D, int HPC>
 static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, cudaStream_t st) {
+                                 const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t st) {
   using L = AttnLayout<D, HPC>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
   static bool configured = false;  // the attribute belongs to the function; set it once
@@ -425,17 +441,18 @@ static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, con
     configured = true;
   }
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hkv * p.n_groups;
-  prefill_attention_kernel<D, HPC><<<grid, AttnRoles<HPC>::kThreads, L::kAlloc, st>>>(tq, tk, tv, p);
+  prefill_attention_kernel<D, HPC><<<grid, AttnRoles<HPC>::kThreads, L::kAlloc, st>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_attention(const AttnParams& p, int D, int hpc, const CUtensorMap& tq,
-                                     const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
-  if (D == 256 && hpc == 1) return launch_attn_t<256, 1>(p, tq, tk, tv, st);
-  if (D == 128 && hpc == 2) return launch_attn_t<128, 2>(p, tq, tk, tv, st);
-  if (D == 128 && hpc == 1) return launch_attn_t<128, 1>(p, tq, tk, tv, st);
-  if (D == 64 && hpc == 2) return launch_attn_t<64, 2>(p, tq, tk, tv, st);
-  if (D == 64 && hpc == 1) return launch_attn_t<64, 1>(p, tq, tk, tv, st);
+                                     const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                                     cudaStream_t st) {
+  if (D == 256 && hpc == 1) return launch_attn_t<256, 1>(p, tq, tk, tv, to, st);
+  if (D == 128 && hpc == 2) return launch_attn_t<128, 2>(p, tq, tk, tv, to, st);
+  if (D == 128 && hpc == 1) return launch_attn_t<128, 1>(p, tq, tk, tv, to, st);
+  if (D == 64 && hpc == 2) return launch_attn_t<64, 2>(p, tq, tk, tv, to, st);
+  if (D == 64 && hpc == 1) return launch_attn_t<64, 1>(p, tq, tk, tv, to, st);
   return cudaErrorInvalidValue;
 }
 
