@@ -17,7 +17,7 @@ Recipe (fixed, documented):
   * every tensor draws from its own CPU torch.Generator seeded with
     seed_for(seed, layer, tensor_id) = 1_000_003*seed + 101*layer + tensor_id
     (tensor ids: q=0, k=1, v=2, q_gamma=3, k_gamma=4, spans=5, lens=6,
-    k_cache=7, v_cache=8);
+    k_cache=7, v_cache=8, dout=9);
   * q, k, v ~ N(0, 1) drawn in fp32 and rounded to bf16;
   * gamma = 1 + 0.1 * N(0, 1), fp32;
   * positions = 0 .. S-1 for every sequence;
@@ -36,7 +36,7 @@ import torch
 LOCAL = 0
 GLOBAL = 1
 
-T_Q, T_K, T_V, T_QG, T_KG, T_SPANS, T_LENS, T_KC, T_VC = range(9)
+T_Q, T_K, T_V, T_QG, T_KG, T_SPANS, T_LENS, T_KC, T_VC, T_DOUT = range(10)
 
 IMAGE_SPAN_TOKENS = 256
 
@@ -156,6 +156,14 @@ def prefill_layer_inputs(B: int, S: int, Hq: int, Hkv: int, D: int, *, seed: int
         positions=positions(B, S),
         spans=image_spans(B, S, n_spans, seed, layer),
     )
+
+
+def prefill_backward_inputs(B: int, S: int, Hq: int, Hkv: int, D: int, *, seed: int = 0,
+                            layer: int = 0, n_spans: int = 0) -> dict:
+    """A layer's prefill inputs plus the output gradient dout [B, S, Hq, D] (bf16, N(0, 1))."""
+    x = prefill_layer_inputs(B, S, Hq, Hkv, D, seed=seed, layer=layer, n_spans=n_spans)
+    x["dout"] = randn_bf16((B, S, Hq, D), seed, layer, T_DOUT)
+    return x
 
 
 def config_layer_inputs(cfg: PrefillConfig, layer: int) -> dict:

@@ -23,3 +23,4 @@ from .attention import (  # noqa: F401
     unmasked_pairs,
 )
 from .projector import soft_tokens  # noqa: F401,E402
+from .backward import prefill_backward, rope_backward, rmsnorm_backward  # noqa: F401,E402
