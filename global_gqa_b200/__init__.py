@@ -46,6 +46,10 @@ _SIGS = {
     "g3attn_prefill_chunk": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_int, _i32,
                                             _f32, _f32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
                                             _sz, _vp]),
+    "g3attn_prefill_backward_workspace_size": (_sz, [_i32] * 5),
+    "g3attn_prefill_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _i32, _f32, _f32, _vp,
+                                               _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _vp, _vp, _vp, _sz, _vp]),
     "g3attn_soft_tokens": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "g3attn_decode_workspace_size": (_sz, [_i32] * 5),
     "g3attn_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, ctypes.c_int, _i32,
@@ -96,6 +100,10 @@ def prefill_workspace_size(B: int, S: int, Hq: int, Hkv: int, D: int) -> int:
 def prefill_chunk_workspace_size(B: int, C: int, Hq: int, Hkv: int, D: int, start: int, layer_kind: int,
                                  window: int) -> int:
     return int(lib().g3attn_prefill_chunk_workspace_size(B, C, Hq, Hkv, D, start, int(layer_kind), window))
+
+
+def prefill_backward_workspace_size(B: int, S: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().g3attn_prefill_backward_workspace_size(B, S, Hq, Hkv, D))
 
 
 def decode_workspace_size(B: int, Hq: int, Hkv: int, D: int, max_seq_len: int) -> int:
@@ -188,6 +196,57 @@ def prefill(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, window: int, 
                               _stream_ptr(stream, q.device))
     _check(st, "g3attn_prefill")
     return (out, lse) if return_lse else out
+
+
+def prefill_backward(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, window: int, rope_base: float,
+                     interp_factor: float, image_spans, out, lse, dout, *, grads=None, ws=None, stream=None):
+    """Gradients of one prefill layer: returns dict(dq, dk, dv, dq_gamma, dk_gamma).
+
+    Arguments as for prefill, plus the forward's out [B,S,Hq,D] bf16 and lse
+    [B,Hq,S] fp32 and the output gradient dout [B,S,Hq,D] bf16.  `grads` may
+    hold preallocated outputs under the same keys.
+    """
+    torch = _torch()
+    _req(q, "q", torch.bfloat16)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _req(k, "k", torch.bfloat16, (B, S, Hkv, D))
+    _req(v, "v", torch.bfloat16, (B, S, Hkv, D))
+    _req(q_gamma, "q_gamma", torch.float32, (D,))
+    _req(k_gamma, "k_gamma", torch.float32, (D,))
+    _req(positions, "positions", torch.int32, (B, S))
+    _req(out, "out", torch.bfloat16, (B, S, Hq, D))
+    _req(lse, "lse", torch.float32, (B, Hq, S))
+    _req(dout, "dout", torch.bfloat16, (B, S, Hq, D))
+    n_spans = 0
+    if image_spans is not None:
+        _req(image_spans, "image_spans", torch.int32)
+        if image_spans.dim() != 3 or image_spans.shape[0] != B or image_spans.shape[2] != 2:
+            raise ValueError("image_spans must be [B, n, 2]")
+        n_spans = int(image_spans.shape[1])
+        if n_spans == 0:
+            image_spans = None
+    g = dict(grads) if grads is not None else {}
+    g.setdefault("dq", torch.empty_like(q))
+    g.setdefault("dk", torch.empty_like(k))
+    g.setdefault("dv", torch.empty_like(v))
+    g.setdefault("dq_gamma", torch.empty_like(q_gamma))
+    g.setdefault("dk_gamma", torch.empty_like(k_gamma))
+    _req(g["dq"], "dq", torch.bfloat16, (B, S, Hq, D))
+    _req(g["dk"], "dk", torch.bfloat16, (B, S, Hkv, D))
+    _req(g["dv"], "dv", torch.bfloat16, (B, S, Hkv, D))
+    _req(g["dq_gamma"], "dq_gamma", torch.float32, (D,))
+    _req(g["dk_gamma"], "dk_gamma", torch.float32, (D,))
+    need = prefill_backward_workspace_size(B, S, Hq, Hkv, D)
+    wsb = ws if ws is not None else workspace(need, q.device, tag="backward")
+    st = lib().g3attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
+                                       int(layer_kind), int(window), float(rope_base), float(interp_factor),
+                                       _ptr(image_spans), n_spans, B, S, Hq, Hkv, D, _ptr(out), _ptr(lse),
+                                       _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                       _ptr(g["dq_gamma"]), _ptr(g["dk_gamma"]), wsb.data_ptr(), wsb.numel(),
+                                       _stream_ptr(stream, q.device))
+    _check(st, "g3attn_prefill_backward")
+    return g
 
 
 def decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, seq_lens, max_seq_len: int,

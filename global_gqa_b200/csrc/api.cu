@@ -198,6 +198,35 @@ bool decode_ws(int B, int Hq, int Hkv, int D, int max_len, DecodeWs* w) {
 
 bool supported_d(int D) { return D == 64 || D == 128 || D == 256; }
 
+// Prefill backward: the forward prologue's buffers, then the padded row data,
+// the key-tile ranges, the fp32 gradients of the rotated q and k, and the
+// per-block gain partials.
+struct BwdWs {
+  PrefillWs f;
+  size_t rowinfo, colmask, kvrange, dq_hat, dk_hat, gpart, total;
+  int S_pad, n_kvtiles;
+};
+bool bwd_ws(int B, int S, int Hq, int Hkv, int D, BwdWs* w) {
+  if (!prefill_ws(B, S, Hq, Hkv, D, &w->f)) return false;
+  w->n_kvtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
+  w->S_pad = w->n_kvtiles * g3::kTileRows;
+  size_t off = w->f.total;
+  w->rowinfo = off;
+  off = align_up(off + (size_t)B * Hq * w->S_pad * 8, 1024);
+  w->colmask = off;
+  off = align_up(off + (size_t)B * w->S_pad * 8, 1024);
+  w->kvrange = off;
+  off = align_up(off + (size_t)B * w->n_kvtiles * 8, 1024);
+  w->dq_hat = off;
+  off = align_up(off + (size_t)B * S * Hq * D * 4, 1024);
+  w->dk_hat = off;
+  off = align_up(off + (size_t)B * S * Hkv * D * 4, 1024);
+  w->gpart = off;
+  off = align_up(off + (size_t)g3::kNormBwdMaxBlocks * 2 * D * 4, 1024);
+  w->total = off;
+  return true;
+}
+
 }  // namespace
 
 void g3::set_last_error(const char* msg) { g_last_error = msg; }
@@ -228,6 +257,12 @@ size_t g3attn_prefill_chunk_workspace_size(int32_t B, int32_t C, int32_t Hq, int
                                            g3_layer_kind layer_kind, int32_t window) {
   ChunkWs w;
   if (!chunk_ws(B, C, Hq, Hkv, D, start, layer_kind, window, &w)) return 0;
+  return w.total;
+}
+
+size_t g3attn_prefill_backward_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D) {
+  BwdWs w;
+  if (!bwd_ws(B, S, Hq, Hkv, D, &w)) return 0;
   return w.total;
 }
 
@@ -490,6 +525,134 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
     e = traced("prefill_ring_write_back", st, [&] { return g3::launch_ring_write_back(rp, D, st); });
     if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk write-back: %s", cudaGetErrorString(e));
   }
+  return G3_OK;
+}
+
+g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v, const float* q_gamma,
+                                  const float* k_gamma, const int32_t* positions, g3_layer_kind layer_kind,
+                                  int32_t window, float rope_base, float interp_factor, const int32_t* image_spans,
+                                  int32_t n_spans, int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                  const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                  float* dq_gamma, float* dk_gamma, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !q_gamma || !k_gamma || !positions || !out || !lse || !dout || !dq || !dk || !dv ||
+      !dq_gamma || !dk_gamma)
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: a required pointer is NULL");
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || D < 1)
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: sizes must be positive (B=%d S=%d Hq=%d Hkv=%d D=%d)", B, S,
+                Hq, Hkv, D);
+  if (Hq % Hkv != 0) return fail(G3_ERR_INVALID_ARG, "prefill backward: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
+  if (layer_kind != G3_LAYER_LOCAL && layer_kind != G3_LAYER_GLOBAL)
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: bad layer kind %d", (int)layer_kind);
+  if (layer_kind == G3_LAYER_LOCAL && window < 1) return fail(G3_ERR_INVALID_ARG, "prefill backward: window < 1");
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base))
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: bad rope_base");
+  if (!(interp_factor > 0.f) || !std::isfinite(interp_factor))
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: bad interp_factor");
+  if (n_spans < 0 || (n_spans > 0 && image_spans == nullptr) || (n_spans == 0 && image_spans != nullptr))
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: image_spans must be NULL iff n_spans == 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return fail(G3_ERR_INVALID_ARG, "prefill backward: bf16 tensors must be 16-byte aligned");
+  if (D != 64 && D != 128)
+    return fail(G3_ERR_UNSUPPORTED, "prefill backward: head_dim %d not built (64, 128)", D);
+  if ((size_t)B * S * Hq * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "prefill backward: problem too large");
+  const int G = Hq / Hkv;
+  const long long n_qtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
+  if (n_qtiles * B * Hq > 0x7fffffffLL) return fail(G3_ERR_UNSUPPORTED, "prefill backward: grid too large");
+
+  BwdWs w;
+  bwd_ws(B, S, Hq, Hkv, D, &w);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(G3_ERR_WORKSPACE, "prefill backward: workspace NULL or not 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(G3_ERR_WORKSPACE, "prefill backward: workspace %zu bytes < required %zu", workspace_bytes, w.total);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* err = reinterpret_cast<int*>(ws);
+
+  // Forward prologue again: intervals, rotation table, normalised and rotated q and k.
+  g3::PrologueParams pp{};
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.q_gamma = q_gamma;
+  pp.k_gamma = k_gamma;
+  pp.positions = positions;
+  pp.spans = image_spans;
+  pp.n_spans = n_spans;
+  pp.B = B;
+  pp.S = S;
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.kind = (int)layer_kind;
+  pp.window = layer_kind == G3_LAYER_LOCAL ? window : S;
+  pp.rope_base = rope_base;
+  pp.interp = interp_factor;
+  for (int f = 0; f < D / 2; ++f) pp.inv_freq[f] = std::pow((double)rope_base, -2.0 * f / D);
+  pp.q_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.f.q_hat);
+  pp.k_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.f.k_hat);
+  pp.lo = reinterpret_cast<int32_t*>(ws + w.f.lo);
+  pp.hi = reinterpret_cast<int32_t*>(ws + w.f.hi);
+  pp.rope_table = reinterpret_cast<float2*>(ws + w.f.table);
+  pp.total = S;
+  pp.err = err;
+
+  g3::BwdParams bp{};
+  bp.q = pp.q;
+  bp.k = pp.k;
+  bp.q_gamma = q_gamma;
+  bp.k_gamma = k_gamma;
+  bp.out = static_cast<const __nv_bfloat16*>(out);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.lse = lse;
+  bp.lo = pp.lo;
+  bp.hi = pp.hi;
+  bp.rope_table = pp.rope_table;
+  bp.rowinfo = reinterpret_cast<float2*>(ws + w.rowinfo);
+  bp.colmask = reinterpret_cast<int2*>(ws + w.colmask);
+  bp.kvrange = reinterpret_cast<int2*>(ws + w.kvrange);
+  bp.dq_hat = reinterpret_cast<float*>(ws + w.dq_hat);
+  bp.dk_hat = reinterpret_cast<float*>(ws + w.dk_hat);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.dq = static_cast<__nv_bfloat16*>(dq);
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.gamma_part = reinterpret_cast<float*>(ws + w.gpart);
+  bp.dq_gamma = dq_gamma;
+  bp.dk_gamma = dk_gamma;
+  bp.err = err;
+  bp.B = B;
+  bp.S = S;
+  bp.S_pad = w.S_pad;
+  bp.Hq = Hq;
+  bp.Hkv = Hkv;
+  bp.G = G;
+  bp.n_qtiles = (int)n_qtiles;
+  bp.n_kvtiles = w.n_kvtiles;
+  const long long norm_blocks = ((long long)B * S + 7) / 8;
+  bp.n_norm_blocks = (int)std::min<long long>(norm_blocks, g3::kNormBwdMaxBlocks);
+  bp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  bp.inv_sqrt_d = (float)(1.0 / std::sqrt((double)D));
+
+  CUtensorMap tq, tdo, tk, tv;
+  if (!make_bshd_map(&tq, pp.q_hat, B, S, Hq, D) || !make_bshd_map(&tdo, dout, B, S, Hq, D) ||
+      !make_bshd_map(&tk, pp.k_hat, B, S, Hkv, D) || !make_bshd_map(&tv, v, B, S, Hkv, D))
+    return fail(G3_ERR_CUDA, "prefill backward: cuTensorMapEncodeTiled unavailable or failed");
+
+  cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill backward: %s", cudaGetErrorString(e));
+  e = traced("prefill_prologue", st, [&] { return g3::launch_prefill_prologue(pp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill backward prologue: %s", cudaGetErrorString(e));
+  e = traced("backward_prep", st, [&] { return g3::launch_bwd_prep(bp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward prep: %s", cudaGetErrorString(e));
+  e = traced("backward_dkdv", st, [&] { return g3::launch_bwd_dkdv(bp, D, tq, tdo, tk, tv, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dk/dv: %s", cudaGetErrorString(e));
+  e = traced("backward_dq", st, [&] { return g3::launch_bwd_dq(bp, D, tq, tdo, tk, tv, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dq: %s", cudaGetErrorString(e));
+  e = traced("backward_norm_rope", st, [&] { return g3::launch_bwd_norm_rope(bp, D, st); });
+  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward norm/rope: %s", cudaGetErrorString(e));
   return G3_OK;
 }
 

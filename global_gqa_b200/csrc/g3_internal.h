@@ -120,6 +120,48 @@ struct SoftTokenParams {
 };
 cudaError_t launch_soft_tokens(const SoftTokenParams& p, cudaStream_t st);
 
+// Prefill backward (gradients of one attention call).  Row data padded to
+// whole 128-row tiles: rowinfo [B, Hq, S_pad] of (lse * log2 e, delta =
+// dout . out), +inf and 0 on padding rows; colmask [B, S_pad] of (lo, hi),
+// never visible on padding rows; kvrange [B, n_kv_tiles] of the first and
+// last query tile that sees each key tile.
+struct BwdParams {
+  const __nv_bfloat16* q;      // raw [B,S,Hq,D]
+  const __nv_bfloat16* k;      // raw [B,S,Hkv,D]
+  const float* q_gamma;
+  const float* k_gamma;
+  const __nv_bfloat16* out;    // forward output [B,S,Hq,D]
+  const __nv_bfloat16* dout;   // [B,S,Hq,D]
+  const float* lse;            // forward [B,Hq,S], natural log
+  const int32_t* lo;           // [B,S]
+  const int32_t* hi;
+  const float2* rope_table;    // [B,S,D/2] (cos, sin)
+  float2* rowinfo;
+  int2* colmask;
+  int2* kvrange;
+  float* dq_hat;               // [B,S,Hq,D] fp32, gradient w.r.t. the rotated, normalised q
+  float* dk_hat;               // [B,S,Hkv,D] fp32
+  __nv_bfloat16* dv;           // [B,S,Hkv,D]
+  __nv_bfloat16* dq;           // [B,S,Hq,D]
+  __nv_bfloat16* dk;           // [B,S,Hkv,D]
+  float* gamma_part;           // [n_norm_blocks, 2, D] per-block gain gradients (q, k)
+  float* dq_gamma;             // [D]
+  float* dk_gamma;             // [D]
+  int* err;
+  int B, S, S_pad, Hq, Hkv, G;
+  int n_qtiles, n_kvtiles;
+  int n_norm_blocks;
+  float scale_log2;            // log2(e) / sqrt(D)
+  float inv_sqrt_d;
+};
+constexpr int kNormBwdMaxBlocks = 148 * 4;
+cudaError_t launch_bwd_prep(const BwdParams& p, int D, cudaStream_t st);
+cudaError_t launch_bwd_dkdv(const BwdParams& p, int D, const CUtensorMap& tm_q, const CUtensorMap& tm_do,
+                            const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
+cudaError_t launch_bwd_dq(const BwdParams& p, int D, const CUtensorMap& tm_q, const CUtensorMap& tm_do,
+                          const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
+cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st);
+
 cudaError_t launch_decode_prologue(const DecodeParams& p, int D, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeParams& p, int D, int grid_chunks, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeParams& p, int D, cudaStream_t st);

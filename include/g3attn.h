@@ -150,6 +150,51 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v,
                                void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------- prefill backward
+ * Bytes of workspace g3attn_prefill_backward needs for these sizes (0 if the
+ * sizes are invalid).  The workspace must be 256-byte aligned.
+ */
+size_t g3attn_prefill_backward_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D);
+
+/*
+ * Prefill backward: gradients of a loss through one g3attn_prefill call, with
+ * respect to the raw q, k, v and both QK-norm gains, given dout = dLoss/dout.
+ * The Gemma 3 Technical Report trains these layers (section 3, distillation;
+ * section 4, quantization-aware training).  The chain rule runs through the
+ * softmax over each row's visible set (the same mask as the forward call), the
+ * grouped-query sharing of k and v, the RoPE rotation and the RMS norm.  The
+ * rotated, normalised q and k are recomputed, not stored.
+ *
+ *   q, k, v, q_gamma, k_gamma, positions, layer_kind, window, rope_base,
+ *   interp_factor, image_spans, n_spans, B, S, Hq, Hkv
+ *              exactly as given to the forward g3attn_prefill call
+ *   D          in {64, 128} (head_dim 256 is not built for the backward:
+ *              G3_ERR_UNSUPPORTED)
+ *   out        bf16 [B, S, Hq, D]  the forward call's output
+ *   lse        fp32 [B, Hq, S]     the forward call's lse (required)
+ *   dout       bf16 [B, S, Hq, D]  gradient of the loss with respect to out
+ *   dq         bf16 [B, S, Hq,  D] gradient with respect to q (written)
+ *   dk, dv     bf16 [B, S, Hkv, D] gradients with respect to k and v (written;
+ *              summed over the Hq / Hkv query heads that share each kv head)
+ *   dq_gamma, dk_gamma  fp32 [D] gradients of the two gains (written; summed
+ *              over every token and head in a fixed order, so repeated calls
+ *              give identical results)
+ *   workspace  >= g3attn_prefill_backward_workspace_size(B, S, Hq, Hkv, D) bytes
+ * All tensors are contiguous and 16-byte aligned; the caller owns every buffer.
+ * Invalid arguments are rejected before any launch; a device-side wait that
+ * times out is reported by g3attn_check_device_error().
+ */
+g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v,
+                                  const float* q_gamma, const float* k_gamma,
+                                  const int32_t* positions,
+                                  g3_layer_kind layer_kind, int32_t window,
+                                  float rope_base, float interp_factor,
+                                  const int32_t* image_spans, int32_t n_spans,
+                                  int32_t B, int32_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                  const void* out, const float* lse, const void* dout,
+                                  void* dq, void* dk, void* dv, float* dq_gamma, float* dk_gamma,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* -------------------------------------------------------------- soft tokens
  * Image soft tokens of the multimodal projector ("Gemma explained: what's new
  * in Gemma 3", 27B printout: RMSNorm over the vision features with eps 1e-6,

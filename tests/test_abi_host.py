@@ -123,6 +123,38 @@ def test_prefill_chunk_workspace_sizes(lib):
     assert glb >= 2048 * 32 * 128 * 2 and glb % 1024 == 0
 
 
+def _backward(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, qg=FAKE, kg=FAKE, pos=FAKE, kind=0, window=1024, base=1e4, interp=1.0,
+             spans=None, n_spans=0, B=1, S=256, Hq=4, Hkv=2, D=128, out=FAKE, lse=FAKE, dout=FAKE, dq=FAKE,
+             dk=FAKE, dv=FAKE, dqg=FAKE, dkg=FAKE, ws=FAKE * 256, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.g3attn_prefill_backward(a["q"], a["k"], a["v"], a["qg"], a["kg"], a["pos"], a["kind"], a["window"],
+                                       a["base"], a["interp"], a["spans"], a["n_spans"], a["B"], a["S"], a["Hq"],
+                                       a["Hkv"], a["D"], a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"],
+                                       a["dqg"], a["dkg"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lse=None), 1), (dict(dout=None), 1), (dict(dq=None), 1), (dict(dk_gamma=None, dkg=None), 1),
+    (dict(B=0), 1), (dict(Hq=3), 1), (dict(kind=5), 1), (dict(window=0), 1), (dict(interp=float("nan")), 1),
+    (dict(n_spans=1), 1), (dict(dv=FAKE + 8), 1), (dict(dout=FAKE + 2), 1),
+    (dict(D=256), 2), (dict(D=96), 2), (dict(ws=None), 3), (dict(ws=FAKE * 256 + 64), 3), (dict(wsb=4096), 3),
+])
+def test_prefill_backward_rejects_on_host(lib, kw, code):
+    kw.pop("dk_gamma", None)
+    assert _backward(lib, **kw) == code
+    assert lib.g3attn_last_error() != b""
+
+
+def test_prefill_backward_workspace_sizes(lib):
+    assert lib.g3attn_prefill_backward_workspace_size(1, 0, 4, 2, 128) == 0
+    fwd = lib.g3attn_prefill_workspace_size(1, 8192, 32, 16, 128)
+    bwd = lib.g3attn_prefill_backward_workspace_size(1, 8192, 32, 16, 128)
+    # the forward buffers plus fp32 gradients of the rotated q and k
+    assert bwd >= fwd + 8192 * (32 + 16) * 128 * 4
+    assert bwd % 1024 == 0
+
+
 def _soft(lib, **kw):
     a = dict(p=FAKE, g=FAKE, B=2, gh=64, gw=64, F=1152, pool=4, out=FAKE, stream=None)
     a.update(kw)

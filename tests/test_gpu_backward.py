@@ -1,0 +1,140 @@
+"""Prefill backward parity: g3attn_prefill_backward against the float64 oracle.
+
+The oracle (oracle/backward.py) applies the chain rule to the plain forward
+definition in float64 from the same bf16 inputs.  The CUDA path recomputes
+the rotated q and k in bf16, feeds P and dS to the tensor cores in bf16 and
+rounds dq, dk, dv to bf16.  Each of those roundings is a relative 2^-9 (about
+2e-3); independent roundings over a sum add in quadrature, and the last bf16
+rounding of the result adds its own 2e-3, so the expected relative L2 error
+is a few 1e-3 (measured: 3e-3 to 4e-3).  The bar is a relative L2 error of
+1e-2 on every gradient (the gains included) and a max error of 2e-2 times the
+largest reference magnitude.
+"""
+import numpy as np
+import pytest
+import torch
+
+import global_gqa_b200 as g3
+import inputs
+from oracle import attention as O
+from oracle import backward as BW
+from gpu_helpers import dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+LOC, GLB = O.LOCAL, O.GLOBAL
+REL_L2 = 1e-2
+MAX_REL = 2e-2
+GAMMA_REL = 1e-2
+
+
+def _cmp(got, ref, what, rel_l2=REL_L2, max_rel=MAX_REL):
+    g = got.detach().double().cpu().numpy() if isinstance(got, torch.Tensor) else np.asarray(got, float)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    scale = max(np.abs(r).max(), 1e-30)
+    err = np.abs(g - r)
+    rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+    print(f"{what}: max {err.max():.3e} (ref max {scale:.3e}), rel L2 {rel:.3e}")
+    assert err.max() <= max_rel * scale, f"{what}: max err {err.max():.3e} > {max_rel} x {scale:.3e}"
+    assert rel <= rel_l2, f"{what}: rel L2 {rel:.3e} > {rel_l2}"
+
+
+def _run(xd, kind, W, base, interp, ws=None):
+    out, lse = g3.prefill(xd["q"], xd["k"], xd["v"], xd["q_gamma"], xd["k_gamma"], xd["positions"], kind, W, base,
+                          interp, xd.get("spans"), return_lse=True)
+    grads = g3.prefill_backward(xd["q"], xd["k"], xd["v"], xd["q_gamma"], xd["k_gamma"], xd["positions"], kind, W,
+                                base, interp, xd.get("spans"), out, lse, xd["dout"], ws=ws)
+    assert g3.check_device_error(g3.workspace(0, dev(), tag="backward")) == 0
+    return grads
+
+
+def _oracle(xc, kind, W, base, interp, kv_heads=None):
+    return BW.prefill_backward(xc["q"], xc["k"], xc["v"], xc["q_gamma"], xc["k_gamma"], xc["positions"], kind, W,
+                               base, interp, xc["dout"], xc.get("spans"), kv_heads=kv_heads)
+
+
+CASES = [
+    # B, S, Hq, Hkv, D, kind, W, n_spans
+    (1, 300, 4, 2, 128, LOC, 128, 0),
+    (2, 700, 4, 2, 128, LOC, 256, 1),
+    (1, 1000, 2, 1, 64, GLB, 1024, 2),
+    (1, 129, 4, 4, 64, GLB, 1024, 0),
+    (1, 600, 8, 2, 128, LOC, 100, 2),
+    (1, 1100, 4, 2, 128, GLB, 1024, 1),
+    (2, 257, 2, 2, 64, LOC, 1024, 0),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}_S{c[1]}_H{c[2]}x{c[3]}_D{c[4]}_k{c[5]}_W{c[6]}_sp{c[7]}"
+                                             for c in CASES])
+def test_backward_matches_oracle(case):
+    B, S, Hq, Hkv, D, kind, W, n_spans = case
+    base, interp = (1e4, 1.0) if kind == LOC else (1e6, 8.0)
+    xc = inputs.prefill_backward_inputs(B, S, Hq, Hkv, D, seed=3, layer=S % 5, n_spans=n_spans)
+    if n_spans == 0:
+        xc["spans"] = None
+    got = _run(to_dev(xc), kind, W, base, interp)
+    ref = _oracle(xc, kind, W, base, interp)
+    for name in ("dq", "dk", "dv"):
+        _cmp(got[name], ref[name], name)
+    for name in ("dq_gamma", "dk_gamma"):
+        _cmp(got[name], ref[name], name, rel_l2=GAMMA_REL, max_rel=GAMMA_REL * 2)
+
+
+def test_backward_single_token():
+    """S = 1: the row sees only itself, so out = v, dv = group sum of dout, dq = dk = 0."""
+    xc = inputs.prefill_backward_inputs(2, 1, 4, 2, 128, seed=4, layer=0)
+    xc["spans"] = None
+    got = _run(to_dev(xc), LOC, 1024, 1e4, 1.0)
+    want = xc["dout"].float().reshape(2, 1, 2, 2, 128).sum(dim=3)
+    assert torch.allclose(got["dv"].float().cpu(), want, atol=2e-2, rtol=1e-2)
+    assert got["dq"].float().abs().max().item() < 1e-3
+    assert got["dk"].float().abs().max().item() < 1e-3
+
+
+def test_backward_window_of_one():
+    """W = 1 without images: every row attends to itself only."""
+    xc = inputs.prefill_backward_inputs(1, 333, 4, 2, 64, seed=6, layer=1)
+    xc["spans"] = None
+    got = _run(to_dev(xc), LOC, 1, 1e4, 1.0)
+    want = xc["dout"].float().reshape(1, 333, 2, 2, 64).sum(dim=3)
+    assert torch.allclose(got["dv"].float().cpu(), want, atol=2e-2, rtol=1e-2)
+    assert got["dq"].float().abs().max().item() < 1e-3
+
+
+def test_backward_is_deterministic():
+    xc = inputs.prefill_backward_inputs(1, 900, 4, 2, 128, seed=8, layer=2, n_spans=1)
+    xd = to_dev(xc)
+    a = _run(xd, GLB, 1024, 1e6, 8.0)
+    b = _run(xd, GLB, 1024, 1e6, 8.0)
+    for name in a:
+        assert torch.equal(a[name], b[name]), name
+
+
+def test_backward_rejects_head_dim_256():
+    xc = inputs.prefill_backward_inputs(1, 64, 2, 1, 256, seed=1, layer=0)
+    xd = to_dev(xc)
+    out, lse = g3.prefill(xd["q"], xd["k"], xd["v"], xd["q_gamma"], xd["k_gamma"], xd["positions"], LOC, 1024, 1e4,
+                          1.0, return_lse=True)
+    with pytest.raises(g3.G3Error):
+        g3.prefill_backward(xd["q"], xd["k"], xd["v"], xd["q_gamma"], xd["k_gamma"], xd["positions"], LOC, 1024,
+                            1e4, 1.0, None, out, lse, xd["dout"])
+
+
+@pytest.mark.parametrize("kind", [LOC, GLB])
+def test_backward_8k_block_shapes(kind):
+    """The 27B-shaped 8K layer (32 / 16 heads, D 128): every gradient of one kv
+    head and its two query heads against the oracle."""
+    B, S, Hq, Hkv, D = 1, 8192, 32, 16, 128
+    W, base, interp = (1024, 1e4, 1.0) if kind == LOC else (1024, 1e6, 8.0)
+    xc = inputs.prefill_backward_inputs(B, S, Hq, Hkv, D, seed=0, layer=0 if kind == LOC else 5)
+    xc["spans"] = None
+    got = _run(to_dev(xc), kind, W, base, interp)
+    kvh = 5
+    ref = _oracle(xc, kind, W, base, interp, kv_heads=[kvh])
+    qh = slice(2 * kvh, 2 * kvh + 2)
+    _cmp(got["dq"][:, :, qh], ref["dq"][:, :, qh], "dq")
+    _cmp(got["dk"][:, :, kvh], ref["dk"][:, :, kvh], "dk")
+    _cmp(got["dv"][:, :, kvh], ref["dv"][:, :, kvh], "dv")
