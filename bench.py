@@ -371,6 +371,91 @@ def run_gpu(args, rank, world, local_rank):
                 "note": "inputs 604 MB > L2, re-read each call"}
         del px, so
 
+    # ---- backward of the block (outside the timed region): every layer's
+    # gradients from its forward out / lse and a random dout
+    backward = None
+    if args.extras:
+        bws = torch.empty(g3.prefill_backward_workspace_size(cfg.B, cfg.S, cfg.Hq, cfg.Hkv, cfg.D),
+                          dtype=torch.uint8, device=dev)
+        fwd = []
+        for li, (L, x) in enumerate(layers):
+            o, lse = g3.prefill(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind,
+                                L.window, L.rope_base, L.interp, x["spans"], return_lse=True, ws=ws, stream=stream)
+            do = torch.empty_like(o)
+            inputs.device_fill_normal_bf16(do, seed=100 + li)
+            fwd.append((o, lse, do))
+        grads = {"dq": torch.empty_like(layers[0][1]["q"]), "dk": torch.empty_like(layers[0][1]["k"]),
+                 "dv": torch.empty_like(layers[0][1]["v"]),
+                 "dq_gamma": torch.empty(cfg.D, dtype=torch.float32, device=dev),
+                 "dk_gamma": torch.empty(cfg.D, dtype=torch.float32, device=dev)}
+
+        def backward_block():
+            for (L, x), (o, lse, do) in zip(layers, fwd):
+                g3.prefill_backward(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind,
+                                    L.window, L.rope_base, L.interp, x["spans"], o, lse, do, grads=grads, ws=bws,
+                                    stream=stream)
+
+        for _ in range(3):
+            backward_block()
+        if g3.check_device_error(bws) != 0:
+            raise RuntimeError("device error in the backward warm-up")
+        reps = max(args.steps // 2, 5)
+        g3.trace_collect()
+        barrier()
+        g3.trace_enable(True)
+        e0b = torch.cuda.Event(enable_timing=True)
+        e1b = torch.cuda.Event(enable_timing=True)
+        e0b.record(stream)
+        for _ in range(reps):
+            backward_block()
+        e1b.record(stream)
+        barrier()
+        g3.trace_enable(False)
+        tr = g3.trace_collect()
+        if g3.check_device_error(bws) != 0:
+            raise RuntimeError("device error in the backward timing")
+        bms = e0b.elapsed_time(e1b) / reps
+        # Algorithmic FLOPs: five products per visible pair (S, dP, dV, dK, dQ)
+        # = 2.5 x the forward's two.  The dK/dV kernel executes four of them
+        # (S^T, dP^T, dV, dK) and the dQ kernel three (S, dP, dQ).
+        alg = 2.5 * block_flops
+        ker = {}
+        for name, mult in (("backward_dkdv", 2.0), ("backward_dq", 1.5)):
+            n_k, m_k = tr.get(name, (0, 0.0))
+            tf = mult * block_flops * reps / (m_k * 1e-3) / 1e12 if m_k > 0 else None
+            ker[name] = {"launches": n_k, "ms": m_k, "tflops_executed": tf,
+                         "frac_of_measured_peak": tf / peak_tf if tf else None}
+        for name in ("prefill_prologue", "backward_prep", "backward_norm_rope"):
+            n_k, m_k = tr.get(name, (0, 0.0))
+            ker[name] = {"launches": n_k, "ms": m_k}
+        kinds = {}
+        for li in (0, len(blk) - 1):
+            (L, x), (o, lse, do) = layers[li], fwd[li]
+            f = metrics.layer_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, L.kind, L.window)
+            g3.trace_collect()
+            barrier()
+            g3.trace_enable(True)
+            for _ in range(5):
+                g3.prefill_backward(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind,
+                                    L.window, L.rope_base, L.interp, x["spans"], o, lse, do, grads=grads, ws=bws,
+                                    stream=stream)
+            barrier()
+            g3.trace_enable(False)
+            tl = g3.trace_collect()
+            row = {}
+            for name, mult in (("backward_dkdv", 2.0), ("backward_dq", 1.5)):
+                n_k, m_k = tl.get(name, (1, 0.0))
+                row[name] = {"us": 1e3 * m_k / n_k, "tflops_executed": mult * f / (m_k / n_k * 1e-3) / 1e12}
+            for name in ("prefill_prologue", "backward_prep", "backward_norm_rope"):
+                n_k, m_k = tl.get(name, (1, 0.0))
+                row[name] = {"us": 1e3 * m_k / n_k}
+            kinds["local" if L.kind == 0 else "global"] = row
+        backward = {"workload": f"{cfg.name}: gradients of all six layers (dq, dk, dv, both gains)",
+                    "ms_per_block": bms, "tflops": alg / (bms * 1e-3) / 1e12,
+                    "flops_per_block": alg, "flops_note": "algorithmic: 2.5 x the forward's unmasked FLOPs",
+                    "kernels": ker, "layer_kinds": kinds}
+        del bws, fwd, grads
+
     # ---- end to end through the public API from pinned host memory
     host = []
     for L, x in layers:
@@ -423,6 +508,7 @@ def run_gpu(args, rank, world, local_rank):
         "chunked_prefill": chunked,
         "shapes_1b": shapes_1b,
         "soft_tokens": soft,
+        "backward": backward,
         "gpu_launches": sum(v[0] for v in trace.values()),
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
