@@ -203,7 +203,7 @@ bool supported_d(int D) { return D == 64 || D == 128 || D == 256; }
 // per-block gain partials.
 struct BwdWs {
   PrefillWs f;
-  size_t rowinfo, colmask, kvrange, dq_hat, dk_hat, gpart, total;
+  size_t lse2, delta, colmask, kvrange, dq_hat, dk_hat, gpart, total;
   int S_pad, n_kvtiles;
 };
 bool bwd_ws(int B, int S, int Hq, int Hkv, int D, BwdWs* w) {
@@ -211,8 +211,10 @@ bool bwd_ws(int B, int S, int Hq, int Hkv, int D, BwdWs* w) {
   w->n_kvtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
   w->S_pad = w->n_kvtiles * g3::kTileRows;
   size_t off = w->f.total;
-  w->rowinfo = off;
-  off = align_up(off + (size_t)B * Hq * w->S_pad * 8, 1024);
+  w->lse2 = off;
+  off = align_up(off + (size_t)B * Hq * w->S_pad * 4, 1024);
+  w->delta = off;
+  off = align_up(off + (size_t)B * Hq * w->S_pad * 4, 1024);
   w->colmask = off;
   off = align_up(off + (size_t)B * w->S_pad * 8, 1024);
   w->kvrange = off;
@@ -608,10 +610,12 @@ g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v, c
   bp.out = static_cast<const __nv_bfloat16*>(out);
   bp.dout = static_cast<const __nv_bfloat16*>(dout);
   bp.lse = lse;
+  bp.q_hat = pp.q_hat;
   bp.lo = pp.lo;
   bp.hi = pp.hi;
   bp.rope_table = pp.rope_table;
-  bp.rowinfo = reinterpret_cast<float2*>(ws + w.rowinfo);
+  bp.lse2 = reinterpret_cast<float*>(ws + w.lse2);
+  bp.delta = reinterpret_cast<float*>(ws + w.delta);
   bp.colmask = reinterpret_cast<int2*>(ws + w.colmask);
   bp.kvrange = reinterpret_cast<int2*>(ws + w.kvrange);
   bp.dq_hat = reinterpret_cast<float*>(ws + w.dq_hat);

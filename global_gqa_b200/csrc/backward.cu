@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(BwdParams p) {
       for (int off = LPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
       if (li == 0 && h < p.Hq) {
         const size_t bh = (size_t)b * p.Hq + h;
-        p.rowinfo[bh * p.S_pad + t] = real ? make_float2(p.lse[bh * p.S + t] * kLog2e, d) : make_float2(INFINITY, 0.f);
+        p.lse2[bh * p.S_pad + t] = real ? p.lse[bh * p.S + t] * kLog2e : INFINITY;
+        p.delta[bh * p.S_pad + t] = d;
       }
     }
   }
@@ -290,16 +291,42 @@ cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st) {
 
 // ================================================================ bwd_dkdv
 // Warp roles of both backward attention kernels: warp 0 TMA producer, warp 1
-// tensor-memory owner and tcgen05.mma issuer, warps 2-9 the elementwise work
-// (two warps per TMEM lane quarter, each on 16 rows; thread t holds rows
-// t/4 and t/4+8 of its slice and columns 8k + 2(t%4) + {0,1}, k < 16).
-constexpr int kBwdThreads = 320;
+// tensor-memory owner and tcgen05.mma issuer, warps 2-17 the elementwise work.
+// The elementwise step needs no row reduction (lse and delta are known), so
+// the 128 columns of a tile are split between two warps: four warps per TMEM
+// lane quarter, each on 16 rows x 64 columns; thread t holds rows t/4 and
+// t/4+8 of its slice and columns 64h + 8k + 2(t%4) + {0,1}, k < 8, of its half h.
+constexpr int kBwdEwWarps = 16;
+constexpr int kBwdThreads = (2 + kBwdEwWarps) * 32;
+constexpr int kBwdEwThreads = kBwdEwWarps * 32;
 constexpr int kBwdFirstWarp = 2;
+
+// Elementwise warp e = warp - 2: TMEM lane quarter warp % 4 (hardware rule),
+// 16-row half (e >> 2) & 1, column half e >> 3.
+__device__ __forceinline__ int bwd_lane_base(int warp) {
+  return (warp & 3) * 32 + (((warp - kBwdFirstWarp) >> 2) & 1) * 16;
+}
+__device__ __forceinline__ int bwd_col_half(int warp) { return (warp - kBwdFirstWarp) >> 3; }
+
+// The bf16 tile a column half packs (P^T, dS^T, dS) goes over the first 32 of
+// its own 64 fp32 columns, so no warp overwrites columns another warp has yet
+// to read: the 16-column (8 TMEM column) chunk kk of the 128 packed columns
+// sits at TMEM column 8 kk + 32 (kk / 4).
+__host__ __device__ constexpr uint32_t bf16_chunk_col(int kk) { return 8 * kk + 32 * (kk / 4); }
+
+// Loads this thread's D/2 columns (half h) of a TMEM accumulator of D columns.
+template <int D>
+__device__ __forceinline__ void tmem_ld_half(uint32_t taddr, float* v) {
+  if constexpr (D == 128) tmem_ld_16x256b_x8(taddr, v);
+  else tmem_ld_16x256b_x4(taddr, v);
+}
 constexpr int kBwdSwizzleBlock = 128 * 64 * 2;  // 128 rows x 64 bf16
 
+constexpr int kBwdMaxStages = 4;
 struct BwdBarriers {
   uint64_t kv_full;
-  uint64_t full[3], empty[3];
+  uint64_t q_ready;  // bwd_dq: Q and dO are in tensor memory
+  uint64_t full[kBwdMaxStages], empty[kBwdMaxStages];
   uint64_t s_full, dp_full, p_full, ds_full, s_free, o_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -310,7 +337,7 @@ template <int D>
 struct DkdvLayout {
   static constexpr int kStages = (D == 64) ? 3 : 2;
   static constexpr int kTile = 128 * D * 2;
-  static constexpr int kSide = 2 * 128 * 8;  // (lse2, delta) then (lo, hi) of the stage's 128 query rows
+  static constexpr int kSide = 2 * 128 * 8;  // lse2, delta, then (lo, hi) of the stage's 128 query rows
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
   static constexpr int kStage0 = kV + kTile;
@@ -320,14 +347,18 @@ struct DkdvLayout {
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-// TMEM columns: S^T (P^T as bf16 over its first 64) at 0, dP^T (dS^T) at 128,
-// dV at 256, dK at 256 + D.
+// TMEM columns: S^T (P^T as bf16 over it) at 0, dP^T (dS^T) at 128, dV at
+// 256, dK at 256 + D.  Per item n the MMA thread issues dV(n) once P^T is
+// stored, then S^T(n+1) (after the dV that read P^T), then dK(n) once dS^T
+// is stored, then dP^T(n+1): the exponentials of item n+1 start while dK(n)
+// and dP^T(n+1) run.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdParams p) {
   using L = DkdvLayout<D>;
   constexpr int NS = L::kStages;
+  static_assert(NS <= kBwdMaxStages && sizeof(BwdBarriers) <= L::kBytes - L::kBar, "barrier block");
   constexpr int KB = D / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -343,21 +374,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int kvh = rem % p.Hkv, b = rem / p.Hkv;
   const int j0 = kt * kTileRows;
   const int2 qr = p.kvrange[(size_t)b * p.n_kvtiles + kt];
-  const int n_items = (qr.y - qr.x + 1) * p.G;  // (query tile, query head of the group)
+  // Items (query tile, query head of the group), query tiles in descending
+  // order: the CTAs of neighbouring key tiles then stream the same query tiles
+  // at the same time and share them in L2.
+  const int n_items = (qr.y - qr.x + 1) * p.G;
   const int n_pre = min(n_items, NS);
 
   auto stage_ptr = [&](int s) { return smem + L::kStage0 + s * L::kStageBytes; };
   auto issue_stage = [&](int n) {
     const int s = n % NS;
     const int h = kvh * p.G + n % p.G;
-    const int q0 = (qr.x + n / p.G) * kTileRows;
+    const int q0 = (qr.y - n / p.G) * kTileRows;
     uint8_t* st = stage_ptr(s);
     mbar_arrive_expect_tx(&bars->full[s], 2 * L::kTile + L::kSide);
     for (int kb = 0; kb < KB; ++kb) {
       tma_load_4d(st + kb * kBwdSwizzleBlock, &tm_q, &bars->full[s], kb * 64, h, q0, b);
       tma_load_4d(st + L::kTile + kb * kBwdSwizzleBlock, &tm_do, &bars->full[s], kb * 64, h, q0, b);
     }
-    bulk_load(st + 2 * L::kTile, p.rowinfo + ((size_t)b * p.Hq + h) * p.S_pad + q0, 1024, &bars->full[s]);
+    const size_t rq = ((size_t)b * p.Hq + h) * p.S_pad + q0;
+    bulk_load(st + 2 * L::kTile, p.lse2 + rq, 512, &bars->full[s]);
+    bulk_load(st + 2 * L::kTile + 512, p.delta + rq, 512, &bars->full[s]);
     bulk_load(st + 2 * L::kTile + 1024, p.colmask + (size_t)b * p.S_pad + q0, 1024, &bars->full[s]);
   };
 
@@ -369,9 +405,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_full, 256);
-    mbar_init(&bars->ds_full, 256);
-    mbar_init(&bars->s_free, 256);
+    mbar_init(&bars->p_full, kBwdEwThreads);
+    mbar_init(&bars->ds_full, kBwdEwThreads);
+    mbar_init(&bars->s_free, kBwdEwThreads);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -396,7 +432,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int last[3] = {-1, -1, -1};
+      int last[kBwdMaxStages] = {-1, -1, -1, -1};
       for (int n = 0; n < n_pre; ++n) last[n] = 0;
       for (int n = n_pre; n < n_items; ++n) {
         const int s = n % NS;
@@ -429,8 +465,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto issue_acc = [&](uint32_t a_col, uint32_t b_addr, uint32_t d_col, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + d_col, tmem + a_col + kk * 8, smem_desc_sw128(b_addr + kk * 2048, kBwdSwizzleBlock, 1024),
-                 idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + d_col, tmem + a_col + bf16_chunk_col(kk),
+                 smem_desc_sw128(b_addr + kk * 2048, kBwdSwizzleBlock, 1024), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
       auto q_addr = [&](int s) { return smem_u32(stage_ptr(s)); };
       auto do_addr = [&](int s) { return smem_u32(stage_ptr(s) + L::kTile); };
@@ -472,35 +508,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ------------------------------------------------------ P^T and dS^T
-    const int lane_base = (warp & 3) * 32 + (((warp - kBwdFirstWarp) >> 2) & 1) * 16;
+    const int lane_base = bwd_lane_base(warp), ch = bwd_col_half(warp);
     const int m4 = lane & 3;
     const int ra = lane_base + (lane >> 2), rb = ra + 8;
     const int ja = j0 + ra, jb = j0 + rb;  // key index of each of this thread's rows
     const uint32_t t_lane = tmem + ((uint32_t)lane_base << 16);
     const float sc = p.scale_log2;
-    const int32_t* lo_b = p.lo + (size_t)b * p.S;
-    const int32_t* hi_b = p.hi + (size_t)b * p.S;
     bool ok = true;
     for (int n = 0; n < n_items; ++n) {
       const int s = n % NS;
-      const int q0 = (qr.x + n / p.G) * kTileRows;
+      const int q0 = (qr.y - n / p.G) * kTileRows;
       const int q_last = min(q0 + kTileRows - 1, p.S - 1);
-      const bool full = lo_b[q_last] <= j0 && hi_b[q0] >= j0 + kTileRows - 1;
-      const float4* ri = reinterpret_cast<const float4*>(stage_ptr(s) + 2 * L::kTile);
-      const int4* cm = reinterpret_cast<const int4*>(stage_ptr(s) + 2 * L::kTile + 1024);
+      // Side data of the stage, per pair of query columns c0 = 64h + 8k + 2 m4, c0 + 1.
+      const float2* l2 = reinterpret_cast<const float2*>(stage_ptr(s) + 2 * L::kTile) + 32 * ch;
+      const float2* dl = reinterpret_cast<const float2*>(stage_ptr(s) + 2 * L::kTile + 512) + 32 * ch;
+      const int2* cm2 = reinterpret_cast<const int2*>(stage_ptr(s) + 2 * L::kTile + 1024);
+      const int4* cm = reinterpret_cast<const int4*>(cm2) + 32 * ch;  // (lo, hi) of two columns per int4
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->full[s], (n / NS) & 1, abort, p.err, 50));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, abort, p.err, 51));
+      if (!ok) break;
+      // Every query row of the tile sees every key of this tile: no mask.
+      const bool full = cm2[q_last - q0].x <= j0 && cm2[0].y >= j0 + kTileRows - 1;
+      float2 lv[8];  // read while S^T is still being computed
+#pragma unroll
+      for (int k = 0; k < 8; ++k) lv[k] = l2[4 * k + m4];
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, abort, p.err, 51));
       if (!ok) break;
       tc_fence_after();
-      float pv[64];
-      tmem_ld_16x256b_x16(t_lane, pv);
+      float pv[32];
+      tmem_ld_16x256b_x8(t_lane + 64 * ch, pv);
       tmem_wait_ld();
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float4 r = ri[4 * k + m4];  // (lse2, delta) of query columns c0 = 8k + 2 m4 and c0 + 1
-        float x0 = fmaf(pv[4 * k], sc, -r.x), x1 = fmaf(pv[4 * k + 1], sc, -r.z);
-        float x2 = fmaf(pv[4 * k + 2], sc, -r.x), x3 = fmaf(pv[4 * k + 3], sc, -r.z);
+      for (int k = 0; k < 8; ++k) {
+        float x0 = fmaf(pv[4 * k], sc, -lv[k].x), x1 = fmaf(pv[4 * k + 1], sc, -lv[k].y);
+        float x2 = fmaf(pv[4 * k + 2], sc, -lv[k].x), x3 = fmaf(pv[4 * k + 3], sc, -lv[k].y);
         if (!full) {
           const int4 c = cm[4 * k + m4];  // (lo, hi) of the two query columns
           if (ja < c.x || ja > c.y) x0 = -INFINITY;
@@ -515,24 +556,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         pk[2 * k] = pack_bf16x2(pv[4 * k], pv[4 * k + 1]);
         pk[2 * k + 1] = pack_bf16x2(pv[4 * k + 2], pv[4 * k + 3]);
       }
-      tmem_st_16x128b_x16(t_lane, pk);
+      tmem_st_16x128b_x8(t_lane + 64 * ch, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
 
+#pragma unroll
+      for (int k = 0; k < 8; ++k) lv[k] = dl[4 * k + m4];  // delta of the two columns
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, n & 1, abort, p.err, 52));
       if (!ok) break;
       tc_fence_after();
-      float dp[64];
-      tmem_ld_16x256b_x16(t_lane + 128, dp);
+      float dp[32];
+      tmem_ld_16x256b_x8(t_lane + 128 + 64 * ch, dp);
       tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float4 r = ri[4 * k + m4];
-        pk[2 * k] = pack_bf16x2(pv[4 * k] * (dp[4 * k] - r.y), pv[4 * k + 1] * (dp[4 * k + 1] - r.w));
-        pk[2 * k + 1] = pack_bf16x2(pv[4 * k + 2] * (dp[4 * k + 2] - r.y), pv[4 * k + 3] * (dp[4 * k + 3] - r.w));
+      for (int k = 0; k < 8; ++k) {
+        pk[2 * k] = pack_bf16x2(pv[4 * k] * (dp[4 * k] - lv[k].x), pv[4 * k + 1] * (dp[4 * k + 1] - lv[k].y));
+        pk[2 * k + 1] = pack_bf16x2(pv[4 * k + 2] * (dp[4 * k + 2] - lv[k].x), pv[4 * k + 3] * (dp[4 * k + 3] - lv[k].y));
       }
-      tmem_st_16x128b_x16(t_lane + 128, pk);
+      tmem_st_16x128b_x8(t_lane + 128 + 64 * ch, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_full);
@@ -540,31 +582,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort, p.err, 53));
     if (ok) {
       tc_fence_after();
+      constexpr int HC = D / 2;  // accumulator columns of this warp
       const bool va = ja < p.S, vb = jb < p.S;
-      __nv_bfloat16* dva = p.dv + ((size_t)(b * p.S + ja) * p.Hkv + kvh) * D;
-      __nv_bfloat16* dvb = p.dv + ((size_t)(b * p.S + jb) * p.Hkv + kvh) * D;
-      float* dka = p.dk_hat + ((size_t)(b * p.S + ja) * p.Hkv + kvh) * D;
-      float* dkb = p.dk_hat + ((size_t)(b * p.S + jb) * p.Hkv + kvh) * D;
+      __nv_bfloat16* dva = p.dv + ((size_t)(b * p.S + ja) * p.Hkv + kvh) * D + HC * ch;
+      __nv_bfloat16* dvb = p.dv + ((size_t)(b * p.S + jb) * p.Hkv + kvh) * D + HC * ch;
+      float* dka = p.dk_hat + ((size_t)(b * p.S + ja) * p.Hkv + kvh) * D + HC * ch;
+      float* dkb = p.dk_hat + ((size_t)(b * p.S + jb) * p.Hkv + kvh) * D + HC * ch;
+      float o[HC / 2];
+      tmem_ld_half<D>(t_lane + 256 + HC * ch, o);
+      tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < D / 64; ++q) {
-        float o[32];
-        tmem_ld_16x256b_x8(t_lane + 256 + q * 64, o);
-        tmem_wait_ld();
+      for (int k = 0; k < HC / 8; ++k) {
+        const int col = 8 * k + 2 * m4;
+        if (va) *reinterpret_cast<uint32_t*>(dva + col) = pack_bf16x2(o[4 * k], o[4 * k + 1]);
+        if (vb) *reinterpret_cast<uint32_t*>(dvb + col) = pack_bf16x2(o[4 * k + 2], o[4 * k + 3]);
+      }
+      tmem_ld_half<D>(t_lane + 256 + D + HC * ch, o);
+      tmem_wait_ld();
+      const float is = p.inv_sqrt_d;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int col = q * 64 + 8 * k + 2 * m4;
-          if (va) *reinterpret_cast<uint32_t*>(dva + col) = pack_bf16x2(o[4 * k], o[4 * k + 1]);
-          if (vb) *reinterpret_cast<uint32_t*>(dvb + col) = pack_bf16x2(o[4 * k + 2], o[4 * k + 3]);
-        }
-        tmem_ld_16x256b_x8(t_lane + 256 + D + q * 64, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int col = q * 64 + 8 * k + 2 * m4;
-          if (va) *reinterpret_cast<float2*>(dka + col) = make_float2(o[4 * k] * p.inv_sqrt_d, o[4 * k + 1] * p.inv_sqrt_d);
-          if (vb)
-            *reinterpret_cast<float2*>(dkb + col) = make_float2(o[4 * k + 2] * p.inv_sqrt_d, o[4 * k + 3] * p.inv_sqrt_d);
-        }
+      for (int k = 0; k < HC / 8; ++k) {
+        const int col = 8 * k + 2 * m4;
+        if (va) *reinterpret_cast<float2*>(dka + col) = make_float2(o[4 * k] * is, o[4 * k + 1] * is);
+        if (vb) *reinterpret_cast<float2*>(dkb + col) = make_float2(o[4 * k + 2] * is, o[4 * k + 3] * is);
       }
     }
   }
@@ -605,27 +645,30 @@ cudaError_t launch_bwd_dkdv(const BwdParams& p, int D, const CUtensorMap& tq, co
 // ================================================================== bwd_dq
 template <int D>
 struct DqLayout {
-  static constexpr int kStages = (D == 64) ? 3 : 2;
+  static constexpr int kStages = (D == 64) ? 4 : 3;
   static constexpr int kTile = 128 * D * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kDO = kQ + kTile;
-  static constexpr int kStage0 = kDO + kTile;
+  static constexpr int kStage0 = 0;
   static constexpr int kStageBytes = 2 * kTile;  // K, V
   static constexpr int kBar = kStage0 + kStages * kStageBytes;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-// TMEM columns: S at 0, dP (dS as bf16 over its first 64) at 128, dQ at 256.
-// Per key tile t the MMA thread issues S(t+1) as soon as the elementwise
-// warps have read S(t), then dQ += dS(t) K(t), then dP(t+1), so the
-// exponentials of tile t+1 overlap the tensor-core work of tile t.
+// TMEM columns: S at 0, dP (dS as bf16 over it) at 128, dQ at 256, and the
+// CTA's Q and dO tiles as bf16 pairs at 384 and 384 + D/2: S = Q K^T and
+// dP = dO V^T read their A operand from tensor memory, so shared memory holds
+// only the K/V ring (three stages at D = 128).  Per key tile t the MMA thread
+// issues S(t+1) as soon as the elementwise warps have read S(t), then
+// dQ += dS(t) K(t), then dP(t+1), so the exponentials of tile t+1 overlap the
+// tensor-core work of tile t.
+constexpr int kDqQCol = 384;
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdParams p) {
   using L = DqLayout<D>;
   constexpr int NS = L::kStages;
+  static_assert(NS <= kBwdMaxStages && sizeof(BwdBarriers) <= L::kBytes - L::kBar, "barrier block");
   constexpr int KB = D / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -659,30 +702,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   };
 
+  // Q and dO into tensor memory: unit u (32 columns = 64 features of Q or
+  // dO) is written by the elementwise warps with u = e >> 2, one row per
+  // thread (the 32x32b shape), as the raw bf16 pairs of the row; rows past S
+  // are zero.  The global loads start before the CTA-wide barrier.
+  constexpr int kUnits = D / 32;
+  const int q_unit = (warp - kBwdFirstWarp) >> 2;
+  const bool q_writer = warp >= kBwdFirstWarp && q_unit < kUnits;
+  const int q_row = (warp & 3) * 32 + lane;
+  uint32_t qw[32];
+  if (q_writer) {
+    const int tensor = q_unit / (D / 64), cb = q_unit % (D / 64);
+    if (r0 + q_row < p.S) {
+      const __nv_bfloat16* src =
+          (tensor == 0 ? p.q_hat : p.dout) + ((size_t)(b * p.S + r0 + q_row) * p.Hq + h) * D + cb * 64;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+        qw[4 * i] = v.x;
+        qw[4 * i + 1] = v.y;
+        qw[4 * i + 2] = v.z;
+        qw[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) qw[i] = 0u;
+    }
+  }
+
   if (tid == 0) {
-    mbar_init(&bars->kv_full, 1);  // here: the Q and dO tiles
+    mbar_init(&bars->q_ready, kBwdEwThreads);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_full, 256);
-    mbar_init(&bars->ds_full, 256);
-    mbar_init(&bars->s_free, 256);
+    mbar_init(&bars->p_full, kBwdEwThreads);
+    mbar_init(&bars->ds_full, kBwdEwThreads);
+    mbar_init(&bars->s_free, kBwdEwThreads);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
-    prefetch_tensormap(&tm_q);
-    prefetch_tensormap(&tm_do);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
-    mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
-    for (int kb = 0; kb < KB; ++kb) {
-      tma_load_4d(smem + L::kQ + kb * kBwdSwizzleBlock, &tm_q, &bars->kv_full, kb * 64, h, r0, b);
-      tma_load_4d(smem + L::kDO + kb * kBwdSwizzleBlock, &tm_do, &bars->kv_full, kb * 64, h, r0, b);
-    }
     for (int t = 0; t < n_pre; ++t) issue_stage(t);
   }
   if (warp == 1) tmem_alloc(&bars->tmem_base, 512);
@@ -694,7 +758,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int last[3] = {-1, -1, -1};
+      int last[kBwdMaxStages] = {-1, -1, -1, -1};
       for (int t = 0; t < n_pre; ++t) last[t] = 0;
       for (int t = n_pre; t < n_tiles; ++t) {
         const int s = t % NS;
@@ -706,32 +770,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       volatile int no_abort = 0;
       for (int s = 0; s < NS; ++s)
         if (last[s] >= 0) mbar_wait(&bars->full[s], last[s], &no_abort, p.err, 61);
-      mbar_wait(&bars->kv_full, 0, &no_abort, p.err, 61);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = smem_u32(smem + L::kQ), do_addr = smem_u32(smem + L::kDO);
-      auto issue_x = [&](uint32_t a_addr, uint32_t b_addr, uint32_t col) {
+      constexpr uint32_t q_col = kDqQCol, do_col = kDqQCol + D / 2;
+      // X = A B^T over the D features: A (Q or dO) from tensor memory, B (K or V) from shared memory.
+      auto issue_x = [&](uint32_t a_col, uint32_t b_addr, uint32_t col) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * kBwdSwizzleBlock + (kk % 4) * 32;
-          mma_ss(tmem + col, smem_desc_sw128(a_addr + off, 16, 1024), smem_desc_sw128(b_addr + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          mma_ts(tmem + col, tmem + a_col + kk * 8, smem_desc_sw128(b_addr + off, 16, 1024), idesc_s,
+                 kk > 0 ? 1u : 0u);
         }
       };
       auto k_addr = [&](int s) { return smem_u32(stage_ptr(s)); };
       auto v_addr = [&](int s) { return smem_u32(stage_ptr(s) + L::kTile); };
 
-      bool ok = mbar_wait(&bars->kv_full, 0, abort, p.err, 62);
+      bool ok = mbar_wait(&bars->q_ready, 0, abort, p.err, 62);
       if (ok) ok = mbar_wait(&bars->full[0], 0, abort, p.err, 63);
       if (ok) {
         tc_fence_after();
-        issue_x(q_addr, k_addr(0), 0);  // S = Q K^T
+        issue_x(q_col, k_addr(0), 0);  // S = Q K^T
         mma_commit(&bars->s_full);
-        issue_x(do_addr, v_addr(0), 128);  // dP = dO V^T
+        issue_x(do_col, v_addr(0), 128);  // dP = dO V^T
         mma_commit(&bars->dp_full);
       }
       for (int t = 0; ok && t < n_tiles; ++t) {
@@ -741,7 +805,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!(ok = mbar_wait(&bars->full[s1], ((t + 1) / NS) & 1, abort, p.err, 64))) break;
           if (!(ok = mbar_wait(&bars->s_free, t & 1, abort, p.err, 65))) break;
           tc_fence_after();
-          issue_x(q_addr, k_addr(s1), 0);
+          issue_x(q_col, k_addr(s1), 0);
           mma_commit(&bars->s_full);
         }
         if (!(ok = mbar_wait(&bars->ds_full, t & 1, abort, p.err, 66))) break;
@@ -750,11 +814,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t kb_addr = k_addr(s);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256, tmem + 128 + kk * 8, smem_desc_sw128(kb_addr + kk * 2048, kBwdSwizzleBlock, 1024),
-                 idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + 256, tmem + 128 + bf16_chunk_col(kk),
+                 smem_desc_sw128(kb_addr + kk * 2048, kBwdSwizzleBlock, 1024), idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[s]);
         if (more) {
-          issue_x(do_addr, v_addr(s1), 128);
+          issue_x(do_col, v_addr(s1), 128);
           mma_commit(&bars->dp_full);
         }
       }
@@ -765,31 +829,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ P and dS
-    const int lane_base = (warp & 3) * 32 + (((warp - kBwdFirstWarp) >> 2) & 1) * 16;
+    const int lane_base = bwd_lane_base(warp), ch = bwd_col_half(warp);
     const int m4 = lane & 3;
     const int ra = lane_base + (lane >> 2), rb = ra + 8;
     const bool valid_a = r0 + ra < p.S, valid_b = r0 + rb < p.S;
     const int lo_a = valid_a ? p.lo[rowbase + r0 + ra] : 1, hi_a = valid_a ? p.hi[rowbase + r0 + ra] : 0;
     const int lo_b = valid_b ? p.lo[rowbase + r0 + rb] : 1, hi_b = valid_b ? p.hi[rowbase + r0 + rb] : 0;
-    const float2 ria = p.rowinfo[((size_t)b * p.Hq + h) * p.S_pad + r0 + ra];  // (lse2, delta); padding: (+inf, 0)
-    const float2 rib = p.rowinfo[((size_t)b * p.Hq + h) * p.S_pad + r0 + rb];
+    const size_t rq = ((size_t)b * p.Hq + h) * p.S_pad + r0;  // padding rows: lse2 +inf, delta 0
+    const float2 ria = make_float2(p.lse2[rq + ra], p.delta[rq + ra]);
+    const float2 rib = make_float2(p.lse2[rq + rb], p.delta[rq + rb]);
     const uint32_t t_lane = tmem + ((uint32_t)lane_base << 16);
     const float sc = p.scale_log2;
+    if (q_writer) {
+      const int tensor = q_unit / (D / 64), cb = q_unit % (D / 64);
+      tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + kDqQCol + tensor * (D / 2) + cb * 32, qw);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(&bars->q_ready);
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, t & 1, abort, p.err, 70));
       if (!ok) break;
       tc_fence_after();
-      float pv[64];
-      tmem_ld_16x256b_x16(t_lane, pv);
+      float pv[32];
+      tmem_ld_16x256b_x8(t_lane + 64 * ch, pv);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bars->s_free);
       const int tile0 = (t_begin + t) * kTileRows;
       const bool full = tile0 >= lo_last && tile0 + kTileRows - 1 <= hi_first;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int col = tile0 + 8 * k + 2 * m4;
+      for (int k = 0; k < 8; ++k) {
+        const int col = tile0 + 64 * ch + 8 * k + 2 * m4;
         float x0 = fmaf(pv[4 * k], sc, -ria.x), x1 = fmaf(pv[4 * k + 1], sc, -ria.x);
         float x2 = fmaf(pv[4 * k + 2], sc, -rib.x), x3 = fmaf(pv[4 * k + 3], sc, -rib.x);
         if (!full) {
@@ -806,16 +878,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, t & 1, abort, p.err, 71));
       if (!ok) break;
       tc_fence_after();
-      float dp[64];
-      tmem_ld_16x256b_x16(t_lane + 128, dp);
+      float dp[32];
+      tmem_ld_16x256b_x8(t_lane + 128 + 64 * ch, dp);
       tmem_wait_ld();
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < 8; ++k) {
         pk[2 * k] = pack_bf16x2(pv[4 * k] * (dp[4 * k] - ria.y), pv[4 * k + 1] * (dp[4 * k + 1] - ria.y));
         pk[2 * k + 1] = pack_bf16x2(pv[4 * k + 2] * (dp[4 * k + 2] - rib.y), pv[4 * k + 3] * (dp[4 * k + 3] - rib.y));
       }
-      tmem_st_16x128b_x16(t_lane + 128, pk);
+      tmem_st_16x128b_x8(t_lane + 128 + 64 * ch, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_full);
@@ -823,22 +895,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort, p.err, 72));
     if (ok) {
       tc_fence_after();
-      float* dqa = p.dq_hat + ((size_t)(b * p.S + r0 + ra) * p.Hq + h) * D;
-      float* dqb = p.dq_hat + ((size_t)(b * p.S + r0 + rb) * p.Hq + h) * D;
+      constexpr int HC = D / 2;
+      float* dqa = p.dq_hat + ((size_t)(b * p.S + r0 + ra) * p.Hq + h) * D + HC * ch;
+      float* dqb = p.dq_hat + ((size_t)(b * p.S + r0 + rb) * p.Hq + h) * D + HC * ch;
+      float o[HC / 2];
+      tmem_ld_half<D>(t_lane + 256 + HC * ch, o);
+      tmem_wait_ld();
+      const float is = p.inv_sqrt_d;
 #pragma unroll
-      for (int q = 0; q < D / 64; ++q) {
-        float o[32];
-        tmem_ld_16x256b_x8(t_lane + 256 + q * 64, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int col = q * 64 + 8 * k + 2 * m4;
-          if (valid_a)
-            *reinterpret_cast<float2*>(dqa + col) = make_float2(o[4 * k] * p.inv_sqrt_d, o[4 * k + 1] * p.inv_sqrt_d);
-          if (valid_b)
-            *reinterpret_cast<float2*>(dqb + col) =
-                make_float2(o[4 * k + 2] * p.inv_sqrt_d, o[4 * k + 3] * p.inv_sqrt_d);
-        }
+      for (int k = 0; k < HC / 8; ++k) {
+        const int col = 8 * k + 2 * m4;
+        if (valid_a) *reinterpret_cast<float2*>(dqa + col) = make_float2(o[4 * k] * is, o[4 * k + 1] * is);
+        if (valid_b) *reinterpret_cast<float2*>(dqb + col) = make_float2(o[4 * k + 2] * is, o[4 * k + 3] * is);
       }
     }
   }

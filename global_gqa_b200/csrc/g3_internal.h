@@ -121,10 +121,10 @@ struct SoftTokenParams {
 cudaError_t launch_soft_tokens(const SoftTokenParams& p, cudaStream_t st);
 
 // Prefill backward (gradients of one attention call).  Row data padded to
-// whole 128-row tiles: rowinfo [B, Hq, S_pad] of (lse * log2 e, delta =
-// dout . out), +inf and 0 on padding rows; colmask [B, S_pad] of (lo, hi),
-// never visible on padding rows; kvrange [B, n_kv_tiles] of the first and
-// last query tile that sees each key tile.
+// whole 128-row tiles: lse2 [B, Hq, S_pad] = lse * log2 e (+inf on padding
+// rows) and delta [B, Hq, S_pad] = dout . out (0 on padding rows); colmask
+// [B, S_pad] of (lo, hi), never visible on padding rows; kvrange [B,
+// n_kv_tiles] of the first and last query tile that sees each key tile.
 struct BwdParams {
   const __nv_bfloat16* q;      // raw [B,S,Hq,D]
   const __nv_bfloat16* k;      // raw [B,S,Hkv,D]
@@ -133,10 +133,12 @@ struct BwdParams {
   const __nv_bfloat16* out;    // forward output [B,S,Hq,D]
   const __nv_bfloat16* dout;   // [B,S,Hq,D]
   const float* lse;            // forward [B,Hq,S], natural log
+  const __nv_bfloat16* q_hat;  // [B,S,Hq,D] normalised, rotated q (recomputed)
   const int32_t* lo;           // [B,S]
   const int32_t* hi;
   const float2* rope_table;    // [B,S,D/2] (cos, sin)
-  float2* rowinfo;
+  float* lse2;
+  float* delta;
   int2* colmask;
   int2* kvrange;
   float* dq_hat;               // [B,S,Hq,D] fp32, gradient w.r.t. the rotated, normalised q
