@@ -635,8 +635,12 @@ g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v, c
   bp.G = G;
   bp.n_qtiles = (int)n_qtiles;
   bp.n_kvtiles = w.n_kvtiles;
-  const long long norm_blocks = ((long long)B * S + 7) / 8;
-  bp.n_norm_blocks = (int)std::min<long long>(norm_blocks, g3::kNormBwdMaxBlocks);
+  // Norm/RoPE backward blocks: query rows and key rows in proportion to Hq : Hkv.
+  const long long norm_blocks = std::max<long long>(2, std::min<long long>(((long long)B * S + 7) / 8 * 2,
+                                                                           g3::kNormBwdMaxBlocks));
+  bp.n_norm_blocks = (int)norm_blocks;
+  bp.n_norm_q_blocks =
+      (int)std::min<long long>(norm_blocks - 1, std::max<long long>(1, norm_blocks * Hq / (Hq + Hkv)));
   bp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   bp.inv_sqrt_d = (float)(1.0 / std::sqrt((double)D));
 

@@ -62,18 +62,24 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
 }  // namespace
 
 // ================================================================ bwd_prep
+// Flat, coalesced pass over the (token, head) rows of out and dout (rows are
+// contiguous in [B, S, Hq, D]): LPR lanes per row, 16-byte loads, kPrepUnroll
+// row steps in flight per warp.  Padding rows, the row intervals (colmask) and
+// the key-tile ranges are grid-stride loops of their own.
+constexpr int kPrepUnroll = 4;
+
 template <int D>
 __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(BwdParams p) {
   constexpr int LPR = D / 8;  // lanes per row, 8 features each
   constexpr int RPW = 32 / LPR;
-  const int lane = threadIdx.x & 31, li = lane % LPR, sub = lane / LPR;
+  const long long gtid = (long long)blockIdx.x * kPrepThreads + threadIdx.x;
+  const long long nthr = (long long)gridDim.x * kPrepThreads;
 
   // Query tiles that see key tile kt: rows i with hi_i >= j0 and lo_i <= j1.
   // Both ends are non-decreasing in i, so these rows are contiguous; row j0
   // itself is one of them.
-  const int gtid = blockIdx.x * kPrepThreads + threadIdx.x;
-  if (gtid < p.B * p.n_kvtiles) {
-    const int b = gtid / p.n_kvtiles, kt = gtid % p.n_kvtiles;
+  for (long long i = gtid; i < (long long)p.B * p.n_kvtiles; i += nthr) {
+    const int b = (int)(i / p.n_kvtiles), kt = (int)(i % p.n_kvtiles);
     const int j0 = kt * kTileRows, j1 = min(j0 + kTileRows - 1, p.S - 1);
     const int32_t* lo = p.lo + (size_t)b * p.S;
     const int32_t* hi = p.hi + (size_t)b * p.S;
@@ -89,47 +95,73 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(BwdParams p) {
       const int m = (l + r + 1) >> 1;
       if (lo[m] <= j1) l = m; else r = m - 1;
     }
-    p.kvrange[gtid] = make_int2(i_min / kTileRows, l / kTileRows);
+    p.kvrange[i] = make_int2(i_min / kTileRows, l / kTileRows);
+  }
+  // Row intervals padded to whole tiles (padding rows see nothing).
+  for (long long i = gtid; i < (long long)p.B * p.S_pad; i += nthr) {
+    const int b = (int)(i / p.S_pad), t = (int)(i % p.S_pad);
+    const size_t src = (size_t)b * p.S + t;
+    p.colmask[i] = t < p.S ? make_int2(p.lo[src], p.hi[src]) : make_int2(0x3fffffff, -1);
+  }
+  // Padding rows of lse2 / delta: P is exactly 0 there.
+  const int pad = p.S_pad - p.S;
+  for (long long i = gtid; i < (long long)p.B * p.Hq * pad; i += nthr) {
+    const long long bh = i / pad;
+    const size_t idx = (size_t)bh * p.S_pad + p.S + (int)(i % pad);
+    p.lse2[idx] = INFINITY;
+    p.delta[idx] = 0.f;
   }
 
-  const int n_tok = p.B * p.S_pad;
-  const int warps_total = gridDim.x * (kPrepThreads / 32);
-  for (int bt = blockIdx.x * (kPrepThreads / 32) + (threadIdx.x >> 5); bt < n_tok; bt += warps_total) {
-    const int b = bt / p.S_pad, t = bt % p.S_pad;
-    const bool real = t < p.S;
-    if (lane == 0) {
-      const size_t src = (size_t)b * p.S + t;
-      p.colmask[bt] = real ? make_int2(p.lo[src], p.hi[src]) : make_int2(0x3fffffff, -1);
-    }
-    for (int h0 = 0; h0 < p.Hq; h0 += RPW) {
-      const int h = h0 + sub;
-      float d = 0.f;
-      if (real && h < p.Hq) {
-        const size_t row = ((size_t)b * p.S + t) * p.Hq + h;
-        float o[8], g[8];
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(p.out + row * D) + li), o);
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + li), g);
+  // Rows in (sequence, head, token) order, token fastest: lse reads and the
+  // lse2 / delta writes are contiguous; each row of out / dout is 2D bytes.
+  const int lane = threadIdx.x & 31, li = lane % LPR, sub = lane / LPR;
+  const long long n_rows = (long long)p.B * p.S * p.Hq;
+  const long long warp_g = gtid >> 5, n_warps = nthr >> 5;
+  for (long long base = warp_g * RPW * kPrepUnroll; base < n_rows; base += n_warps * RPW * kPrepUnroll) {
+    uint4 o[kPrepUnroll], g[kPrepUnroll];
+    float l[kPrepUnroll];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d = fmaf(o[e], g[e], d);
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      const long long row = base + u * RPW + sub;  // = (b * Hq + h) * S + t
+      if (row < n_rows) {
+        const long long bh = row / p.S;
+        const int t = (int)(row % p.S);
+        const int b = (int)(bh / p.Hq), h = (int)(bh % p.Hq);
+        const size_t src = ((size_t)(b * p.S + t) * p.Hq + h) * D;
+        o[u] = __ldg(reinterpret_cast<const uint4*>(p.out + src) + li);
+        g[u] = __ldg(reinterpret_cast<const uint4*>(p.dout + src) + li);
+        l[u] = li == 0 ? __ldg(p.lse + row) : 0.f;
+      } else {
+        o[u] = g[u] = make_uint4(0u, 0u, 0u, 0u);
+        l[u] = 0.f;
       }
+    }
+#pragma unroll
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      float a[8], c[8];
+      bf16x8_to_f32(o[u], a);
+      bf16x8_to_f32(g[u], c);
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) d = fmaf(a[e], c[e], d);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      if (li == 0 && h < p.Hq) {
-        const size_t bh = (size_t)b * p.Hq + h;
-        p.lse2[bh * p.S_pad + t] = real ? p.lse[bh * p.S + t] * kLog2e : INFINITY;
-        p.delta[bh * p.S_pad + t] = d;
+      const long long row = base + u * RPW + sub;
+      if (li == 0 && row < n_rows) {
+        const size_t idx = (size_t)(row / p.S) * p.S_pad + (int)(row % p.S);
+        p.lse2[idx] = l[u] * kLog2e;
+        p.delta[idx] = d;
       }
     }
   }
 }
 
 cudaError_t launch_bwd_prep(const BwdParams& p, int D, cudaStream_t st) {
-  const long long warps = (long long)p.B * p.S_pad;
-  long long blocks = (warps + 7) / 8;
-  const long long kv_blocks = ((long long)p.B * p.n_kvtiles + kPrepThreads - 1) / kPrepThreads;
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
-  if (blocks < kv_blocks) blocks = kv_blocks;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long rows = (long long)p.B * p.S * p.Hq;
+  const int rpw = 32 / (D / 8);
+  long long blocks = (rows + (long long)rpw * kPrepUnroll * 8 - 1) / ((long long)rpw * kPrepUnroll * 8);
+  if (blocks > 148LL * 8) blocks = 148LL * 8;
+  if (blocks < 1) blocks = 1;
   switch (D) {
     case 64: bwd_prep_kernel<64><<<(unsigned)blocks, kPrepThreads, 0, st>>>(p); break;
     case 128: bwd_prep_kernel<128><<<(unsigned)blocks, kPrepThreads, 0, st>>>(p); break;
@@ -141,9 +173,13 @@ cudaError_t launch_bwd_prep(const BwdParams& p, int D, cudaStream_t st) {
 // =========================================================== bwd_norm_rope
 // One warp per token; lane li of a row holds features d1 .. d1+7 and
 // D/2+d1 .. D/2+d1+7 (rotation partners together), as in the forward pass.
-// Row h < Hq is query head h, else key head h - Hq.
+// The first n_norm_q_blocks blocks take the query rows, the others the key
+// rows, so each lane accumulates the gradient of one gain only; kNormUnroll
+// row steps are in flight per warp.
+constexpr int kNormUnroll = 2;
+
 template <int D>
-__global__ void __launch_bounds__(kNormThreads) bwd_norm_rope_kernel(BwdParams p) {
+__global__ void __launch_bounds__(kNormThreads, 2) bwd_norm_rope_kernel(BwdParams p) {
   constexpr int H2 = D / 2;
   constexpr int LPR = D / 16;
   constexpr int RPW = 32 / LPR;
@@ -151,18 +187,30 @@ __global__ void __launch_bounds__(kNormThreads) bwd_norm_rope_kernel(BwdParams p
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int li = lane % LPR, sub = lane / LPR;
   const int d1 = li * 8;
-  const int heads = p.Hq + p.Hkv;
+  const bool is_q = (int)blockIdx.x < p.n_norm_q_blocks;
+  const int blk = is_q ? (int)blockIdx.x : (int)blockIdx.x - p.n_norm_q_blocks;
+  const int n_blk = is_q ? p.n_norm_q_blocks : p.n_norm_blocks - p.n_norm_q_blocks;
+  const int heads = is_q ? p.Hq : p.Hkv;
+  const __nv_bfloat16* xsrc = is_q ? p.q : p.k;
+  const float* gsrc = is_q ? p.dq_hat : p.dk_hat;
+  __nv_bfloat16* dst = is_q ? p.dq : p.dk;
   const int n_tokens = p.B * p.S;
-  __shared__ __align__(16) float gam[2 * D];
-  __shared__ float red[NW][2][D];
-  for (int i = threadIdx.x; i < 2 * D; i += kNormThreads) gam[i] = i < D ? p.q_gamma[i] : p.k_gamma[i - D];
+  __shared__ __align__(16) float gam[D];
+  __shared__ float red[NW][D];
+  for (int i = threadIdx.x; i < D; i += kNormThreads) gam[i] = is_q ? p.q_gamma[i] : p.k_gamma[i];
   __syncthreads();
-
-  float acc_q[16], acc_k[16];
+  float gv[16];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) acc_q[e] = acc_k[e] = 0.f;
+  for (int e = 0; e < 8; ++e) {
+    gv[e] = gam[d1 + e];
+    gv[8 + e] = gam[H2 + d1 + e];
+  }
 
-  for (int bt = blockIdx.x * NW + warp; bt < n_tokens; bt += gridDim.x * NW) {
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+
+  for (int bt = blk * NW + warp; bt < n_tokens; bt += n_blk * NW) {
     const float4* tab = reinterpret_cast<const float4*>(p.rope_table + (size_t)bt * H2 + d1);
     float c[8], s[8];
 #pragma unroll
@@ -173,95 +221,93 @@ __global__ void __launch_bounds__(kNormThreads) bwd_norm_rope_kernel(BwdParams p
       c[2 * i + 1] = v.z;
       s[2 * i + 1] = v.w;
     }
-    for (int h0 = 0; h0 < heads; h0 += RPW) {
-      const int h = h0 + sub;
-      const bool valid = h < heads;
-      const bool is_q = h < p.Hq;
-      float x[16], g[16];
-      if (valid) {
-        const __nv_bfloat16* src = is_q ? p.q + ((size_t)bt * p.Hq + h) * D : p.k + ((size_t)bt * p.Hkv + h - p.Hq) * D;
-        const float* gsrc =
-            is_q ? p.dq_hat + ((size_t)bt * p.Hq + h) * D : p.dk_hat + ((size_t)bt * p.Hkv + h - p.Hq) * D;
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(src + d1)), x);
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(src + H2 + d1)), x + 8);
+    for (int h0 = 0; h0 < heads; h0 += RPW * kNormUnroll) {
+      uint4 xa[kNormUnroll], xb[kNormUnroll];
+      float4 ga[kNormUnroll][2], gb[kNormUnroll][2];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          *reinterpret_cast<float4*>(g + 4 * i) = __ldg(reinterpret_cast<const float4*>(gsrc + d1) + i);
-          *reinterpret_cast<float4*>(g + 8 + 4 * i) = __ldg(reinterpret_cast<const float4*>(gsrc + H2 + d1) + i);
+      for (int u = 0; u < kNormUnroll; ++u) {
+        const int h = h0 + u * RPW + sub;
+        if (h < heads) {
+          const size_t row = (size_t)bt * heads + h;
+          xa[u] = __ldg(reinterpret_cast<const uint4*>(xsrc + row * D + d1));
+          xb[u] = __ldg(reinterpret_cast<const uint4*>(xsrc + row * D + H2 + d1));
+          ga[u][0] = __ldg(reinterpret_cast<const float4*>(gsrc + row * D + d1));
+          ga[u][1] = __ldg(reinterpret_cast<const float4*>(gsrc + row * D + d1) + 1);
+          gb[u][0] = __ldg(reinterpret_cast<const float4*>(gsrc + row * D + H2 + d1));
+          gb[u][1] = __ldg(reinterpret_cast<const float4*>(gsrc + row * D + H2 + d1) + 1);
+        } else {
+          xa[u] = xb[u] = make_uint4(0u, 0u, 0u, 0u);
+          ga[u][0] = ga[u][1] = gb[u][0] = gb[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) x[e] = g[e] = 0.f;
-      }
-      // Inverse rotation: the gradient of y = R(theta) x is R(theta)^T dy.
-      float gt[16];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        gt[e] = g[e] * c[e] + g[8 + e] * s[e];
-        gt[8 + e] = g[8 + e] * c[e] - g[e] * s[e];
-      }
-      const float* gm = gam + (is_q ? 0 : D);
-      float gv[16];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        gv[e] = gm[d1 + e];
-        gv[8 + e] = gm[H2 + d1 + e];
-      }
-      float ss = 0.f, inner = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        ss = fmaf(x[e], x[e], ss);
-        inner = fmaf(gv[e] * gt[e], x[e], inner);
       }
 #pragma unroll
-      for (int off = LPR / 2; off > 0; off >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        inner += __shfl_xor_sync(0xffffffffu, inner, off);
-      }
-      if (!valid) continue;
-      // y = x r gamma, r = (mean x^2 + eps)^(-1/2), as in the forward pass.
-      const float r = rsqrtf(ss * (1.0f / D) + 1e-6f);
-      const float t3 = r * r * r * inner * (1.0f / D);
-      float dx[16];
+      for (int u = 0; u < kNormUnroll; ++u) {
+        const int h = h0 + u * RPW + sub;
+        float x[16], g[16];
+        bf16x8_to_f32(xa[u], x);
+        bf16x8_to_f32(xb[u], x + 8);
+        *reinterpret_cast<float4*>(g) = ga[u][0];
+        *reinterpret_cast<float4*>(g + 4) = ga[u][1];
+        *reinterpret_cast<float4*>(g + 8) = gb[u][0];
+        *reinterpret_cast<float4*>(g + 12) = gb[u][1];
+        // Inverse rotation: the gradient of y = R(theta) x is R(theta)^T dy.
+        float gt[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        dx[e] = r * gv[e] * gt[e] - x[e] * t3;
-        if (is_q) acc_q[e] = fmaf(gt[e] * r, x[e], acc_q[e]);
-        else acc_k[e] = fmaf(gt[e] * r, x[e], acc_k[e]);
+        for (int e = 0; e < 8; ++e) {
+          gt[e] = g[e] * c[e] + g[8 + e] * s[e];
+          gt[8 + e] = g[8 + e] * c[e] - g[e] * s[e];
+        }
+        float ss = 0.f, inner = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          ss = fmaf(x[e], x[e], ss);
+          inner = fmaf(gv[e] * gt[e], x[e], inner);
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) {
+          ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          inner += __shfl_xor_sync(0xffffffffu, inner, off);
+        }
+        if (h >= heads) continue;
+        // y = x r gamma, r = (mean x^2 + eps)^(-1/2), as in the forward pass.
+        const float r = rsqrtf(ss * (1.0f / D) + 1e-6f);
+        const float t3 = r * r * r * inner * (1.0f / D);
+        float dx[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          dx[e] = r * gv[e] * gt[e] - x[e] * t3;
+          acc[e] = fmaf(gt[e] * r, x[e], acc[e]);
+        }
+        __nv_bfloat16* o = dst + ((size_t)bt * heads + h) * D;
+        *reinterpret_cast<uint4*>(o + d1) = make_uint4(pack_bf16x2(dx[0], dx[1]), pack_bf16x2(dx[2], dx[3]),
+                                                       pack_bf16x2(dx[4], dx[5]), pack_bf16x2(dx[6], dx[7]));
+        *reinterpret_cast<uint4*>(o + H2 + d1) =
+            make_uint4(pack_bf16x2(dx[8], dx[9]), pack_bf16x2(dx[10], dx[11]), pack_bf16x2(dx[12], dx[13]),
+                       pack_bf16x2(dx[14], dx[15]));
       }
-      __nv_bfloat16* dst = is_q ? p.dq + ((size_t)bt * p.Hq + h) * D : p.dk + ((size_t)bt * p.Hkv + h - p.Hq) * D;
-      *reinterpret_cast<uint4*>(dst + d1) =
-          make_uint4(pack_bf16x2(dx[0], dx[1]), pack_bf16x2(dx[2], dx[3]), pack_bf16x2(dx[4], dx[5]),
-                     pack_bf16x2(dx[6], dx[7]));
-      *reinterpret_cast<uint4*>(dst + H2 + d1) =
-          make_uint4(pack_bf16x2(dx[8], dx[9]), pack_bf16x2(dx[10], dx[11]), pack_bf16x2(dx[12], dx[13]),
-                     pack_bf16x2(dx[14], dx[15]));
     }
   }
-  // Gains: lanes with the same features (same li) combine, then the warps in
-  // a fixed order; one partial row per block.
+  // Gain: lanes with the same features (same li) combine, then the warps in a
+  // fixed order; one partial row per block (the other gain's row is zero).
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
-      acc_q[e] += __shfl_xor_sync(0xffffffffu, acc_q[e], off);
-      acc_k[e] += __shfl_xor_sync(0xffffffffu, acc_k[e], off);
-    }
+    for (int off = LPR; off < 32; off <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
   }
   if (sub == 0) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      red[warp][0][d1 + e] = acc_q[e];
-      red[warp][0][H2 + d1 + e] = acc_q[8 + e];
-      red[warp][1][d1 + e] = acc_k[e];
-      red[warp][1][H2 + d1 + e] = acc_k[8 + e];
+      red[warp][d1 + e] = acc[e];
+      red[warp][H2 + d1 + e] = acc[8 + e];
     }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < 2 * D; i += kNormThreads) {
     float sum = 0.f;
+    if ((i < D) == is_q) {
 #pragma unroll
-    for (int w = 0; w < NW; ++w) sum += red[w][i / D][i % D];
+      for (int w = 0; w < NW; ++w) sum += red[w][i % D];
+    }
     p.gamma_part[(size_t)blockIdx.x * 2 * D + i] = sum;
   }
 }
@@ -277,7 +323,9 @@ __global__ void bwd_gamma_reduce_kernel(BwdParams p, int D) {
 }
 
 cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st) {
-  if (p.n_norm_blocks < 1 || p.n_norm_blocks > kNormBwdMaxBlocks) return cudaErrorInvalidValue;
+  if (p.n_norm_blocks < 2 || p.n_norm_blocks > kNormBwdMaxBlocks || p.n_norm_q_blocks < 1 ||
+      p.n_norm_q_blocks >= p.n_norm_blocks)
+    return cudaErrorInvalidValue;
   switch (D) {
     case 64: bwd_norm_rope_kernel<64><<<p.n_norm_blocks, kNormThreads, 0, st>>>(p); break;
     case 128: bwd_norm_rope_kernel<128><<<p.n_norm_blocks, kNormThreads, 0, st>>>(p); break;

@@ -152,7 +152,8 @@ struct BwdParams {
   int* err;
   int B, S, S_pad, Hq, Hkv, G;
   int n_qtiles, n_kvtiles;
-  int n_norm_blocks;
+  int n_norm_blocks;           // blocks of bwd_norm_rope (>= 2)
+  int n_norm_q_blocks;         // the first ones take the query rows, the rest the key rows
   float scale_log2;            // log2(e) / sqrt(D)
   float inv_sqrt_d;
 };
