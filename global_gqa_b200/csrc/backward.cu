@@ -114,23 +114,27 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(BwdParams p) {
 
   // Rows in (sequence, head, token) order, token fastest: lse reads and the
   // lse2 / delta writes are contiguous; each row of out / dout is 2D bytes.
+  // A warp takes a chunk of RPW x kPrepUnroll consecutive tokens of one
+  // (sequence, head).
+  constexpr int kChunk = RPW * kPrepUnroll;
   const int lane = threadIdx.x & 31, li = lane % LPR, sub = lane / LPR;
-  const long long n_rows = (long long)p.B * p.S * p.Hq;
+  const int chunks_per_bh = (p.S + kChunk - 1) / kChunk;
+  const long long n_chunks = (long long)p.B * p.Hq * chunks_per_bh;
   const long long warp_g = gtid >> 5, n_warps = nthr >> 5;
-  for (long long base = warp_g * RPW * kPrepUnroll; base < n_rows; base += n_warps * RPW * kPrepUnroll) {
+  for (long long c = warp_g; c < n_chunks; c += n_warps) {
+    const int bh = (int)(c / chunks_per_bh);
+    const int t0 = (int)(c - (long long)bh * chunks_per_bh) * kChunk;
+    const int b = bh / p.Hq, h = bh - b * p.Hq;
     uint4 o[kPrepUnroll], g[kPrepUnroll];
     float l[kPrepUnroll];
 #pragma unroll
     for (int u = 0; u < kPrepUnroll; ++u) {
-      const long long row = base + u * RPW + sub;  // = (b * Hq + h) * S + t
-      if (row < n_rows) {
-        const long long bh = row / p.S;
-        const int t = (int)(row % p.S);
-        const int b = (int)(bh / p.Hq), h = (int)(bh % p.Hq);
+      const int t = t0 + u * RPW + sub;
+      if (t < p.S) {
         const size_t src = ((size_t)(b * p.S + t) * p.Hq + h) * D;
         o[u] = __ldg(reinterpret_cast<const uint4*>(p.out + src) + li);
         g[u] = __ldg(reinterpret_cast<const uint4*>(p.dout + src) + li);
-        l[u] = li == 0 ? __ldg(p.lse + row) : 0.f;
+        l[u] = li == 0 ? __ldg(p.lse + (size_t)bh * p.S + t) : 0.f;
       } else {
         o[u] = g[u] = make_uint4(0u, 0u, 0u, 0u);
         l[u] = 0.f;
@@ -138,17 +142,17 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(BwdParams p) {
     }
 #pragma unroll
     for (int u = 0; u < kPrepUnroll; ++u) {
-      float a[8], c[8];
+      float a[8], e8[8];
       bf16x8_to_f32(o[u], a);
-      bf16x8_to_f32(g[u], c);
+      bf16x8_to_f32(g[u], e8);
       float d = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) d = fmaf(a[e], c[e], d);
+      for (int e = 0; e < 8; ++e) d = fmaf(a[e], e8[e], d);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      const long long row = base + u * RPW + sub;
-      if (li == 0 && row < n_rows) {
-        const size_t idx = (size_t)(row / p.S) * p.S_pad + (int)(row % p.S);
+      const int t = t0 + u * RPW + sub;
+      if (li == 0 && t < p.S) {
+        const size_t idx = (size_t)bh * p.S_pad + t;
         p.lse2[idx] = l[u] * kLog2e;
         p.delta[idx] = d;
       }
@@ -312,14 +316,39 @@ __global__ void __launch_bounds__(kNormThreads, 2) bwd_norm_rope_kernel(BwdParam
   }
 }
 
-// Sum of the per-block partials in block order.
-__global__ void bwd_gamma_reduce_kernel(BwdParams p, int D) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= 2 * D) return;
+// Sum of the per-block partials: one CTA per 32 columns; warp w sums blocks
+// w, w + 8, ... in eight interleaved partial sums (loads in flight), then the
+// eight warps' sums are added in warp order.  The order is fixed, so repeated
+// calls give identical results.
+constexpr int kGammaWarps = 8;
+__global__ void __launch_bounds__(kGammaWarps * 32) bwd_gamma_reduce_kernel(BwdParams p, int D) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int i = blockIdx.x * 32 + lane;  // column of the [2, D] partial row
+  __shared__ float part[kGammaWarps][32];
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  if (i < 2 * D) {
+    for (int blk0 = warp; blk0 < p.n_norm_blocks; blk0 += 8 * kGammaWarps) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int blk = blk0 + k * kGammaWarps;
+        if (blk < p.n_norm_blocks) acc[k] += p.gamma_part[(size_t)blk * 2 * D + i];
+      }
+    }
+  }
   float sum = 0.f;
-  for (int blk = 0; blk < p.n_norm_blocks; ++blk) sum += p.gamma_part[(size_t)blk * 2 * D + i];
-  if (i < D) p.dq_gamma[i] = sum;
-  else p.dk_gamma[i - D] = sum;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) sum += acc[k];
+  part[warp][lane] = sum;
+  __syncthreads();
+  if (warp == 0 && i < 2 * D) {
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kGammaWarps; ++w) tot += part[w][lane];
+    if (i < D) p.dq_gamma[i] = tot;
+    else p.dk_gamma[i - D] = tot;
+  }
 }
 
 cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st) {
@@ -333,7 +362,7 @@ cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st) {
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_gamma_reduce_kernel<<<(2 * D + 127) / 128, 128, 0, st>>>(p, D);
+  bwd_gamma_reduce_kernel<<<(2 * D + 31) / 32, kGammaWarps * 32, 0, st>>>(p, D);
   return cudaGetLastError();
 }
 
