@@ -403,7 +403,9 @@ constexpr int kBwdMaxStages = 4;
 struct BwdBarriers {
   uint64_t kv_full;
   uint64_t q_ready;  // bwd_dq: Q and dO are in tensor memory
-  uint64_t full[kBwdMaxStages], empty[kBwdMaxStages];
+  // A stage's tiles land on two barriers: full (Q and the side data, or K)
+  // and full2 (dO, or V), so the first product waits for half of the stage.
+  uint64_t full[kBwdMaxStages], full2[kBwdMaxStages], empty[kBwdMaxStages];
   uint64_t s_full, dp_full, p_full, ds_full, s_free, o_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -463,21 +465,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int h = kvh * p.G + n % p.G;
     const int q0 = (qr.y - n / p.G) * kTileRows;
     uint8_t* st = stage_ptr(s);
-    mbar_arrive_expect_tx(&bars->full[s], 2 * L::kTile + L::kSide);
-    for (int kb = 0; kb < KB; ++kb) {
-      tma_load_4d(st + kb * kBwdSwizzleBlock, &tm_q, &bars->full[s], kb * 64, h, q0, b);
-      tma_load_4d(st + L::kTile + kb * kBwdSwizzleBlock, &tm_do, &bars->full[s], kb * 64, h, q0, b);
-    }
+    mbar_arrive_expect_tx(&bars->full[s], L::kTile + L::kSide);
+    for (int kb = 0; kb < KB; ++kb) tma_load_4d(st + kb * kBwdSwizzleBlock, &tm_q, &bars->full[s], kb * 64, h, q0, b);
     const size_t rq = ((size_t)b * p.Hq + h) * p.S_pad + q0;
     bulk_load(st + 2 * L::kTile, p.lse2 + rq, 512, &bars->full[s]);
     bulk_load(st + 2 * L::kTile + 512, p.delta + rq, 512, &bars->full[s]);
     bulk_load(st + 2 * L::kTile + 1024, p.colmask + (size_t)b * p.S_pad + q0, 1024, &bars->full[s]);
+    mbar_arrive_expect_tx(&bars->full2[s], L::kTile);
+    for (int kb = 0; kb < KB; ++kb)
+      tma_load_4d(st + L::kTile + kb * kBwdSwizzleBlock, &tm_do, &bars->full2[s], kb * 64, h, q0, b);
   };
 
   if (tid == 0) {
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->full2[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
@@ -520,7 +523,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       volatile int no_abort = 0;
       for (int s = 0; s < NS; ++s)
-        if (last[s] >= 0) mbar_wait(&bars->full[s], last[s], &no_abort, p.err, 41);
+        if (last[s] >= 0) {
+          mbar_wait(&bars->full[s], last[s], &no_abort, p.err, 41);
+          mbar_wait(&bars->full2[s], last[s], &no_abort, p.err, 41);
+        }
       mbar_wait(&bars->kv_full, 0, &no_abort, p.err, 41);
     }
   } else if (warp == 1) {
@@ -554,6 +560,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         issue_t(k_addr, q_addr(0), 0);
         mma_commit(&bars->s_full);
+      }
+      if (ok) ok = mbar_wait(&bars->full2[0], 0, abort, p.err, 43);
+      if (ok) {
+        tc_fence_after();
         issue_t(v_addr, do_addr(0), 128);
         mma_commit(&bars->dp_full);
       }
@@ -574,6 +584,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_acc(128, q_addr(s), 256 + D, n > 0);  // dK += dS^T Q
         mma_commit(&bars->empty[s]);
         if (more) {
+          if (!(ok = mbar_wait(&bars->full2[s1], ((n + 1) / NS) & 1, abort, p.err, 48))) break;
+          tc_fence_after();
           issue_t(v_addr, do_addr(s1), 128);  // next dP^T (after the dK that read dS^T)
           mma_commit(&bars->dp_full);
         }
@@ -772,11 +784,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto issue_stage = [&](int t) {
     const int s = t % NS;
     const int kv0 = (t_begin + t) * kTileRows;
-    mbar_arrive_expect_tx(&bars->full[s], 2 * L::kTile);
-    for (int kb = 0; kb < KB; ++kb) {
+    mbar_arrive_expect_tx(&bars->full[s], L::kTile);
+    for (int kb = 0; kb < KB; ++kb)
       tma_load_4d(stage_ptr(s) + kb * kBwdSwizzleBlock, &tm_k, &bars->full[s], kb * 64, kvh, kv0, b);
-      tma_load_4d(stage_ptr(s) + L::kTile + kb * kBwdSwizzleBlock, &tm_v, &bars->full[s], kb * 64, kvh, kv0, b);
-    }
+    mbar_arrive_expect_tx(&bars->full2[s], L::kTile);
+    for (int kb = 0; kb < KB; ++kb)
+      tma_load_4d(stage_ptr(s) + L::kTile + kb * kBwdSwizzleBlock, &tm_v, &bars->full2[s], kb * 64, kvh, kv0, b);
   };
 
   // Q and dO into tensor memory: unit u (32 columns = 64 features of Q or
@@ -811,6 +824,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&bars->q_ready, kBwdEwThreads);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->full2[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
@@ -846,7 +860,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       volatile int no_abort = 0;
       for (int s = 0; s < NS; ++s)
-        if (last[s] >= 0) mbar_wait(&bars->full[s], last[s], &no_abort, p.err, 61);
+        if (last[s] >= 0) {
+          mbar_wait(&bars->full[s], last[s], &no_abort, p.err, 61);
+          mbar_wait(&bars->full2[s], last[s], &no_abort, p.err, 61);
+        }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
@@ -872,6 +889,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         issue_x(q_col, k_addr(0), 0);  // S = Q K^T
         mma_commit(&bars->s_full);
+      }
+      if (ok) ok = mbar_wait(&bars->full2[0], 0, abort, p.err, 63);
+      if (ok) {
+        tc_fence_after();
         issue_x(do_col, v_addr(0), 128);  // dP = dO V^T
         mma_commit(&bars->dp_full);
       }
@@ -895,6 +916,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                  smem_desc_sw128(kb_addr + kk * 2048, kBwdSwizzleBlock, 1024), idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[s]);
         if (more) {
+          if (!(ok = mbar_wait(&bars->full2[s1], ((t + 1) / NS) & 1, abort, p.err, 68))) break;
+          tc_fence_after();
           issue_x(do_col, v_addr(s1), 128);
           mma_commit(&bars->dp_full);
         }
