@@ -180,6 +180,41 @@ def oracle_prefill_sample(cfg, budget_s: float, seed: int = 0):
             return flops, secs, nrows
 
 
+def oracle_extras_baselines(line: dict) -> None:
+    """The oracles of the backward and of the soft tokens, timed as they stand
+    on bounded samples of the same workloads (rank 0, N = 1)."""
+    from oracle import backward as BW
+    from oracle import projector as PJ
+    cfg = inputs.BLOCK_8K
+    if line.get("backward"):
+        L = cfg.block()[0]
+        S1 = 2048  # the oracle's cost grows as S^2: the first 2048 tokens of the layer
+        x = inputs.prefill_backward_inputs(cfg.B, S1, cfg.Hq, cfg.Hkv, cfg.D, seed=cfg.seed, layer=0)
+        G = cfg.Hq // cfg.Hkv
+        t0 = time.perf_counter()
+        BW.prefill_backward(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind, L.window,
+                            L.rope_base, L.interp, x["dout"], None, kv_heads=[0])
+        secs = time.perf_counter() - t0
+        flops = 2.5 * metrics.layer_flops(cfg.B, S1, cfg.Hq, cfg.D, L.kind, L.window) * G / cfg.Hq
+        line["backward"]["cpu_baseline"] = {
+            "value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "seconds": secs, "sample": f"gradients of kv head 0 and its {G} query heads over the first {S1} tokens "
+                                       f"of a local layer (W={L.window}) of {cfg.name} (algorithmic FLOPs), "
+                                       f"float64 numpy"}
+    if line.get("soft_tokens"):
+        Bi, gh, F = 8, 64, 1152
+        px = np.random.default_rng(17).standard_normal((Bi, gh * gh, F)).astype(np.float32)
+        gam = np.ones(F)
+        t0 = time.perf_counter()
+        PJ.soft_tokens(px, gam, gh, gh, 4)
+        secs = time.perf_counter() - t0
+        nbytes = (Bi * gh * gh * F + Bi * (gh // 4) ** 2 * F) * 2 + F * 4
+        line["soft_tokens"]["cpu_baseline"] = {
+            "value": nbytes / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle", "seconds": secs,
+            "sample": f"{Bi} of the 64 images (64x64 patches x 1152 features, bytes counted as bf16 like the GPU "
+                      f"metric), float64 numpy"}
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -639,6 +674,8 @@ def main():
                                 "kind": "oracle", "seconds": s,
                                 "sample": f"{r} query rows (groups of 64 per layer, all 32 heads) of the "
                                           f"{inputs.BLOCK_8K.name} block, float64 numpy"}
+        if args.extras and args.cpu_budget > 0:
+            oracle_extras_baselines(line)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
