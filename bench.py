@@ -500,21 +500,50 @@ def run_gpu(args, rank, world, local_rank):
     h2d = sum(v.numel() * v.element_size() for _, hx in host for k, v in hx.items() if v is not None and k != "out")
     d2h = sum(hx["out"].numel() * hx["out"].element_size() for _, hx in host)
 
+    # Uploads, layers and downloads on three streams ordered by events, so a
+    # layer's download overlaps the next layer's upload (the host link is full
+    # duplex) and both overlap the kernels.  A layer's input buffers are
+    # overwritten only after its previous prefill read them, and its output
+    # only after its previous download.
+    h2d_st = torch.cuda.Stream(dev)
+    d2h_st = torch.cuda.Stream(dev)
+    ev_c = [None] * len(layers)
+    ev_d = [None] * len(layers)
+
     def e2e_step():
-        for (L, hx), (_, x) in zip(host, layers):
-            for k in ("q", "k", "v", "q_gamma", "k_gamma", "positions"):
-                x[k].copy_(hx[k], non_blocking=True)
+        for i, ((L, hx), (_, x)) in enumerate(zip(host, layers)):
+            with torch.cuda.stream(h2d_st):
+                if ev_c[i] is not None:
+                    h2d_st.wait_event(ev_c[i])
+                for k in ("q", "k", "v", "q_gamma", "k_gamma", "positions"):
+                    x[k].copy_(hx[k], non_blocking=True)
+                eh = torch.cuda.Event()
+                eh.record(h2d_st)
+            stream.wait_event(eh)
+            if ev_d[i] is not None:
+                stream.wait_event(ev_d[i])
             g3.prefill(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind, L.window,
                        L.rope_base, L.interp, x["spans"], out=x["out"], ws=ws, stream=stream)
-            hx["out"].copy_(x["out"], non_blocking=True)
+            ec = torch.cuda.Event()
+            ec.record(stream)
+            ev_c[i] = ec
+            with torch.cuda.stream(d2h_st):
+                d2h_st.wait_event(ec)
+                hx["out"].copy_(x["out"], non_blocking=True)
+                ed = torch.cuda.Event()
+                ed.record(d2h_st)
+                ev_d[i] = ed
 
     e2e_steps = max(1, min(args.steps, 20))
     e2e_step()
     barrier()
     w0 = time.perf_counter()
     e0.record(stream)
+    h2d_st.wait_event(e0)
     for _ in range(e2e_steps):
         e2e_step()
+    for ed in ev_d:
+        stream.wait_event(ed)
     e1.record(stream)
     barrier()
     wall = time.perf_counter() - w0
