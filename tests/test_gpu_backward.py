@@ -83,6 +83,33 @@ def test_backward_matches_oracle(case):
         _cmp(got[name], ref[name], name, rel_l2=GAMMA_REL, max_rel=GAMMA_REL * 2)
 
 
+EDGE_CASES = [
+    # B, S, Hq, Hkv, D, kind, W, spans (per sequence), positions "shifted" (3t + 7) or None
+    (3, 513, 8, 1, 64, LOC, 37, [[5, 40], [200, 456], [500, 513]], None),
+    (1, 2049, 4, 2, 128, GLB, 1024, [[1000, 1256], [1900, 2049]], None),
+    (2, 700, 4, 2, 128, LOC, 256, [[100, 356]], "shifted"),
+    (1, 128, 4, 4, 64, LOC, 4096, [], None),
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=[f"B{c[0]}_S{c[1]}_H{c[2]}x{c[3]}_D{c[4]}_k{c[5]}_W{c[6]}"
+                                                  f"_sp{len(c[7])}_{c[8] or 'pos'}" for c in EDGE_CASES])
+def test_backward_edge_cases(case):
+    """GQA 8:1, a window of 37, spans touching S, positions that are not 0..S-1, W > S."""
+    B, S, Hq, Hkv, D, kind, W, spans, pos = case
+    base, interp = (1e4, 1.0) if kind == LOC else (1e6, 8.0)
+    xc = inputs.prefill_backward_inputs(B, S, Hq, Hkv, D, seed=21, layer=S % 3)
+    xc["spans"] = torch.tensor([spans] * B, dtype=torch.int32) if spans else None
+    if pos == "shifted":
+        xc["positions"] = (3 * torch.arange(S, dtype=torch.int32) + 7).repeat(B, 1).contiguous()
+    got = _run(to_dev(xc), kind, W, base, interp)
+    ref = _oracle(xc, kind, W, base, interp)
+    for name in ("dq", "dk", "dv"):
+        _cmp(got[name], ref[name], name)
+    for name in ("dq_gamma", "dk_gamma"):
+        _cmp(got[name], ref[name], name, rel_l2=GAMMA_REL, max_rel=GAMMA_REL * 2)
+
+
 def test_backward_single_token():
     """S = 1: the row sees only itself, so out = v, dv = group sum of dout, dq = dk = 0."""
     xc = inputs.prefill_backward_inputs(2, 1, 4, 2, 128, seed=4, layer=0)
