@@ -2,8 +2,8 @@
 // gradients of a loss with respect to the raw q, k, v and the two QK-norm
 // gains, given dout = dLoss/dout and the forward's out and lse.
 //
-// The Gemma 3 Technical Report trains these layers (section 3 "Pre-training",
-// distillation; section 4, quantization-aware training); the forward steps
+// The Gemma 3 Technical Report trains these layers (section 2.2 "Pre-training",
+// distillation; section 2.3 "Quantization Aware Training"); the forward steps
 // are QK-norm and RoPE (section 2 "Model Architecture", "Long context"), the
 // 5:1 local/global mask with bidirectional image spans (sections 1 and 2;
 // "Gemma explained: what's new in Gemma 3", section "Vision encoder and
@@ -62,10 +62,10 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
 }  // namespace
 
 // ================================================================ bwd_prep
-// Flat, coalesced pass over the (token, head) rows of out and dout (rows are
-// contiguous in [B, S, Hq, D]): LPR lanes per row, 16-byte loads, kPrepUnroll
-// row steps in flight per warp.  Padding rows, the row intervals (colmask) and
-// the key-tile ranges are grid-stride loops of their own.
+// Rows of out and dout taken as chunks of consecutive tokens of one (sequence,
+// head): LPR lanes per row, 16-byte loads, kPrepUnroll row steps in flight per
+// warp.  Padding rows, the row intervals (colmask) and the key-tile ranges are
+// grid-stride loops of their own.
 constexpr int kPrepUnroll = 4;
 
 template <int D>

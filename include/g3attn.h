@@ -159,8 +159,8 @@ size_t g3attn_prefill_backward_workspace_size(int32_t B, int32_t S, int32_t Hq, 
 /*
  * Prefill backward: gradients of a loss through one g3attn_prefill call, with
  * respect to the raw q, k, v and both QK-norm gains, given dout = dLoss/dout.
- * The Gemma 3 Technical Report trains these layers (section 3, distillation;
- * section 4, quantization-aware training).  The chain rule runs through the
+ * The Gemma 3 Technical Report trains these layers (section 2.2, distillation;
+ * section 2.3, quantization-aware training).  The chain rule runs through the
  * softmax over each row's visible set (the same mask as the forward call), the
  * grouped-query sharing of k and v, the RoPE rotation and the RMS norm.  The
  * rotated, normalised q and k are recomputed, not stored.

@@ -8,8 +8,8 @@ The forward computation is the one in `oracle.attention` (QK-norm, RoPE, the
 visibility mask, GQA, softmax attention; Gemma 3 Technical Report, section 2
 "Model Architecture" and "Long context"; "Gemma explained: what's new in
 Gemma 3", the q_norm/k_norm lines and section "Vision encoder and
-processing").  The Technical Report trains these layers (section 3,
-"Pre-training": distillation; section 4: quantization-aware training), which
+processing").  The Technical Report trains these layers (section 2.2
+"Pre-training": distillation; section 2.3 "Quantization Aware Training"), which
 needs the gradient of a loss through every one of those steps.  Given
 dout = dLoss/dout, this module applies the chain rule to each forward step in
 reverse order:
