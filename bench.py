@@ -47,9 +47,13 @@ def peaks():
         return dict(FALLBACK), "fallback"
 
 
-def kernel_source_hash() -> str:
+DECODE_TRAFFIC_PATH = os.path.join(ROOT, "profiles", "decode_split_traffic.json")
+
+
+def kernel_source_hash(files=("prefill.cu", "sm100_ptx.cuh", "g3_internal.h")) -> str:
+    """Hash of the sources a committed ncu traffic figure was taken on."""
     h = hashlib.sha256()
-    for f in ("prefill.cu", "sm100_ptx.cuh", "g3_internal.h"):
+    for f in files:
         with open(os.path.join(ROOT, "global_gqa_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -178,6 +182,20 @@ def oracle_prefill_sample(cfg, budget_s: float, seed: int = 0):
         g += 1
         if secs >= budget_s:
             return flops, secs, nrows
+
+
+def decode_traffic_per_launch(alg_bytes_per_launch: float):
+    """DRAM bytes per decode_split launch: the committed capture of a smaller
+    decode (8 sequences of 16K-32K tokens, larger than L2) scaled by algorithmic
+    KV bytes, while the decode sources are the ones it was taken on."""
+    try:
+        with open(DECODE_TRAFFIC_PATH) as f:
+            tr = json.load(f)
+        if tr.get("source_hash") == kernel_source_hash(("decode.cu", "sm100_ptx.cuh", "g3_internal.h")):
+            return tr["bytes_per_algorithmic_byte"] * alg_bytes_per_launch
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
 
 
 def oracle_extras_baselines(line: dict) -> None:
@@ -642,7 +660,8 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
         "config": {"workload": cfg.name, "batch": cfg.B, "context": f"U[{cfg.len_lo},{cfg.len_hi}]",
                    "kv_bytes_per_step": step_bytes, "l2": "inputs larger than L2 (~38 GB of cache read per step)"},
         "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": (ach / pk["hbm_gbs"]) if ach else None, "traffic": None, "kernel": "decode_split",
+                     "frac": (ach / pk["hbm_gbs"]) if ach else None,
+                     "traffic": decode_traffic_per_launch(step_bytes / len(blk)), "kernel": "decode_split",
                      "peak_kind": f"{pk_kind} copy bandwidth", "launches": n_split},
         "kernels": {k: {"launches": v[0], "ms": v[1]} for k, v in trace.items()},
         "gpu_launches": sum(v[0] for v in trace.values()),

@@ -184,3 +184,28 @@ def test_decode_full_size_sampled():
         assert_close(out[check], ref, what=f"decode layer {li}")
         del kc, vc
         torch.cuda.empty_cache()
+
+
+def test_decode_medium_global():
+    """8 sequences of 16K-32K tokens on a global layer (~2 GB of cache, larger than
+    L2): the DRAM traffic of this call is what the decode profile scales; three
+    sequences are checked against the oracle."""
+    B, Hq, Hkv, D, cap = 8, 32, 16, 128, 32768
+    lens = inputs.decode_lengths(B, 16384, cap, seed=3)
+    sl = lens.to(dev())
+    kc = torch.empty(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev())
+    vc = torch.empty_like(kc)
+    inputs.device_fill_normal_bf16(kc, 31)
+    inputs.device_fill_normal_bf16(vc, 32)
+    x = inputs.decode_step_inputs(B, Hq, Hkv, D, seed=3, layer=5)
+    xd = to_dev(x)
+    out = g3.decode(xd["q"], xd["k_new"], xd["v_new"], xd["q_gamma"], xd["k_gamma"], kc, vc, sl, cap, O.GLOBAL,
+                    cap, 1e6, 8.0)
+    assert g3.check_device_error(g3.workspace(0, dev())) == 0
+    check = [0, 3, 7]
+    hk = [kc[b][:, :int(lens[b]) - 1].permute(1, 0, 2).cpu() for b in check]
+    hv = [vc[b][:, :int(lens[b]) - 1].permute(1, 0, 2).cpu() for b in check]
+    sub = {k: v[check] for k, v in x.items() if k in ("q", "k_new", "v_new")}
+    ref, _ = O.decode(sub["q"], sub["k_new"], sub["v_new"], x["q_gamma"], x["k_gamma"], lens[check].numpy(), hk, hv,
+                      [0] * len(check), O.GLOBAL, cap, 1e6, 8.0)
+    assert_close(out[check], ref, what="decode medium")
