@@ -350,7 +350,7 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   pp.k_hat = reinterpret_cast<__nv_bfloat16*>(ws + w.k_hat);
   pp.lo = reinterpret_cast<int32_t*>(ws + w.lo);
   pp.hi = reinterpret_cast<int32_t*>(ws + w.hi);
-  pp.rope_table = reinterpret_cast<float2*>(ws + w.table);
+  pp.rope_table = nullptr;  // the forward pass needs no stored table
   pp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
   pp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
   pp.cache_cap = cache_capacity;
@@ -467,7 +467,7 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
   pp.k_hat = nullptr;  // keys go straight to their rows in `keys`
   pp.lo = reinterpret_cast<int32_t*>(ws + w.lo);
   pp.hi = reinterpret_cast<int32_t*>(ws + w.hi);
-  pp.rope_table = reinterpret_cast<float2*>(ws + w.table);
+  pp.rope_table = nullptr;  // the forward pass needs no stored table
   pp.k_cache = keys;
   pp.v_cache = vals;
   pp.cache_cap = rows;

@@ -34,7 +34,7 @@ struct PrologueParams {
   __nv_bfloat16* k_hat;  // [B,S,Hkv,D]
   int32_t* lo;           // [B,S] first visible key of each row
   int32_t* hi;           // [B,S] last visible key of each row
-  float2* rope_table;    // [B,S,D/2] (cos, sin) of each rotation angle
+  float2* rope_table;    // optional output [B,S,D/2]: (cos, sin) of each rotation angle (NULL: not stored)
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   int cache_cap;

@@ -1,17 +1,18 @@
 // Prefill prologue: QK-RMSNorm + RoPE of q and k, the per-row visible key
-// interval, and the optional KV-cache fill, in two launches:
+// interval, and the optional KV-cache fill, in one launch:
 //
-//   rope_table  : per token, (cos, sin) of every rotation angle, formed and
-//                 evaluated in double and stored as fp32 [B, S, D/2] (a few MB,
-//                 read back from L2); the token's visible interval; validation
-//                 of the image spans.
 //   qk_norm_rope: bandwidth-bound pass over every (token, head) row of q and k.
-//                 One warp per token: the token's cos/sin are loaded once into
-//                 registers and serve all of its Hq + Hkv rows; each lane
-//                 holds 8 features of each half of a row (16-byte accesses,
-//                 rotation partners in the same lane), two row steps in
-//                 flight per warp and 32 warps per SM; the gains are read
-//                 from shared memory to keep registers free.
+//                 One warp per token: the warp forms the token's rotation
+//                 angles and their cos/sin in double (each lane a few of the
+//                 D/2 angles, then shuffles), which serve all of its Hq + Hkv
+//                 rows; lane 0 writes the token's visible interval and, on
+//                 token 0, validates the image spans.  Each lane holds 8
+//                 features of each half of a row (16-byte accesses, rotation
+//                 partners in the same lane), two row steps in flight per warp
+//                 and 32 warps per SM; the gains are read from shared memory to
+//                 keep registers free.  When a table is given (the backward
+//                 pass reads it), the fp32 (cos, sin) of every angle is also
+//                 stored as [B, S, D/2].
 //
 // Norm (Gemma 3 Technical Report, section 2; eps and dim from the q_norm /
 // k_norm lines of "Gemma explained: what's new in Gemma 3"): x / sqrt(mean(x^2)
@@ -36,58 +37,8 @@
 
 namespace g3 {
 
-constexpr int kTableThreads = 256;
 constexpr int kRowThreads = 256;  // 8 warps, one token each at a time
 constexpr int kRowUnroll = 2;     // row steps in flight per warp (32 warps per SM)
-
-template <int D>
-__global__ void __launch_bounds__(kTableThreads) rope_table_kernel(PrologueParams p) {
-  constexpr int H2 = D / 2;
-  __shared__ double inv_freq_s[H2];
-  if (threadIdx.x < H2) inv_freq_s[threadIdx.x] = p.inv_freq[threadIdx.x];
-  __syncthreads();
-  const size_t idx = (size_t)blockIdx.x * kTableThreads + threadIdx.x;
-  const size_t total = (size_t)p.B * p.S * H2;
-  if (idx >= total) return;
-  const size_t bt = idx / H2;
-  const int f = (int)(idx % H2);
-  const int b = (int)(bt / p.S), t = (int)(bt % p.S);
-  const double theta = (double)p.positions[bt] / p.interp * inv_freq_s[f];
-  double sd, cd;
-  sincos(theta, &sd, &cd);
-  p.rope_table[idx] = make_float2((float)cd, (float)sd);
-
-  if (f == 0) {
-    // Interval of token ta (whole-sequence index), as key rows from key_base.
-    const int ta = p.start + t;
-    int lo = (p.kind == 1) ? 0 : max(0, ta - p.window + 1);
-    int hi = ta;
-    const int32_t* sp = p.spans + (size_t)b * p.n_spans * 2;
-    for (int k = 0; k < p.n_spans; ++k) {
-      const int st = sp[2 * k], en = sp[2 * k + 1];
-      if (st <= ta && ta < en) {
-        lo = min(lo, max(st, 0));
-        hi = max(hi, min(en, p.total) - 1);
-        break;
-      }
-    }
-    p.lo[bt] = lo - p.key_base;
-    p.hi[bt] = hi - p.key_base;
-    if (t == 0 && p.n_spans > 0) {
-      // Sorted, disjoint, inside the sequence, and (chunked prefill) not
-      // holding tokens on both sides of the chunk's first or last boundary.
-      int prev_end = 0;
-      bool ok = true;
-      for (int k = 0; k < p.n_spans; ++k) {
-        const int st = sp[2 * k], en = sp[2 * k + 1];
-        ok = ok && st >= prev_end && st < en && en <= p.total;
-        ok = ok && !(st < p.start && en > p.start) && !(st < p.total && en > p.total);
-        prev_end = en;
-      }
-      if (!ok) record_error(p.err, kErrInvalid, 100);
-    }
-  }
-}
 
 __device__ __forceinline__ void unpack4_bf16(const uint2 u, float* f) {
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
@@ -113,20 +64,71 @@ __global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(ProloguePa
   const int heads = p.Hq + p.Hkv;
   const int n_tokens = p.B * p.S;
   const int warps_total = gridDim.x * (kRowThreads / 32);
+  constexpr int FPL = (H2 + 31) / 32;  // rotation angles formed per lane (FPL divides 8)
   __shared__ __align__(16) float gam[2 * D];  // q gain, then k gain
+  __shared__ double inv_freq_s[H2];
   for (int i = threadIdx.x; i < 2 * D; i += kRowThreads) gam[i] = i < D ? p.q_gamma[i] : p.k_gamma[i - D];
+  for (int i = threadIdx.x; i < H2; i += kRowThreads) inv_freq_s[i] = p.inv_freq[i];
   __syncthreads();
 
   for (int bt = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5); bt < n_tokens; bt += warps_total) {
-    const float4* tab = reinterpret_cast<const float4*>(p.rope_table + (size_t)bt * H2 + d1);
+    // Angles (p / interp) * base^(-2f/D) and their cos/sin in double; lane L
+    // forms f = FPL * L .. FPL * L + FPL - 1.
+    float cl[FPL], sl[FPL];
+    const double pos = (double)p.positions[bt] / p.interp;
+#pragma unroll
+    for (int i = 0; i < FPL; ++i) {
+      const int f = FPL * lane + i;
+      cl[i] = 1.f;
+      sl[i] = 0.f;
+      if (f < H2) {
+        double sd, cd;
+        sincos(pos * inv_freq_s[f], &sd, &cd);
+        cl[i] = (float)cd;
+        sl[i] = (float)sd;
+        if (p.rope_table != nullptr) p.rope_table[(size_t)bt * H2 + f] = make_float2(cl[i], sl[i]);
+      }
+    }
+    // This lane's features d1 + e (and their partners) use angle d1 + e, held by
+    // lane (d1 + e) / FPL in slot e % FPL (d1 is a multiple of 8).
     float c[8], s[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 v = __ldg(tab + i);
-      c[2 * i] = v.x;
-      s[2 * i] = v.y;
-      c[2 * i + 1] = v.z;
-      s[2 * i + 1] = v.w;
+    for (int e = 0; e < 8; ++e) {
+      c[e] = __shfl_sync(0xffffffffu, cl[e % FPL], (d1 + e) / FPL);
+      s[e] = __shfl_sync(0xffffffffu, sl[e % FPL], (d1 + e) / FPL);
+    }
+    if (lane == 0) {
+      // Visible interval of token ta (whole-sequence index), as key rows from
+      // key_base: the causal window (or [0, ta] on a global layer) joined with
+      // the token's image span, which is contiguous because both contain ta.
+      const int b = bt / p.S, t = bt % p.S;
+      const int ta = p.start + t;
+      int lo = (p.kind == 1) ? 0 : max(0, ta - p.window + 1);
+      int hi = ta;
+      const int32_t* sp = p.spans + (size_t)b * p.n_spans * 2;
+      for (int k = 0; k < p.n_spans; ++k) {
+        const int st = sp[2 * k], en = sp[2 * k + 1];
+        if (st <= ta && ta < en) {
+          lo = min(lo, max(st, 0));
+          hi = max(hi, min(en, p.total) - 1);
+          break;
+        }
+      }
+      p.lo[bt] = lo - p.key_base;
+      p.hi[bt] = hi - p.key_base;
+      if (t == 0 && p.n_spans > 0) {
+        // Sorted, disjoint, inside the sequence, and (chunked prefill) not
+        // holding tokens on both sides of the chunk's first or last boundary.
+        int prev_end = 0;
+        bool ok = true;
+        for (int k = 0; k < p.n_spans; ++k) {
+          const int st = sp[2 * k], en = sp[2 * k + 1];
+          ok = ok && st >= prev_end && st < en && en <= p.total;
+          ok = ok && !(st < p.start && en > p.start) && !(st < p.total && en > p.total);
+          prev_end = en;
+        }
+        if (!ok) record_error(p.err, kErrInvalid, 100);
+      }
     }
     const __nv_bfloat16* qrow = p.q + (size_t)bt * p.Hq * D;
     const __nv_bfloat16* krow = p.k + (size_t)bt * p.Hkv * D;
@@ -210,19 +212,14 @@ __global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(ProloguePa
 }
 
 cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st) {
-  const size_t table_threads = (size_t)p.B * p.S * (D / 2);
-  const unsigned table_blocks = (unsigned)((table_threads + kTableThreads - 1) / kTableThreads);
   const long long tokens = (long long)p.B * p.S;
   long long blocks = (tokens + (kRowThreads / 32) - 1) / (kRowThreads / 32);
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (D == 128) {
-    rope_table_kernel<128><<<table_blocks, kTableThreads, 0, st>>>(p);
     qk_norm_rope_kernel<128><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
   } else if (D == 64) {
-    rope_table_kernel<64><<<table_blocks, kTableThreads, 0, st>>>(p);
     qk_norm_rope_kernel<64><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
   } else if (D == 256) {
-    rope_table_kernel<256><<<table_blocks, kTableThreads, 0, st>>>(p);
     qk_norm_rope_kernel<256><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
   } else {
     return cudaErrorInvalidValue;
