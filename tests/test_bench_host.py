@@ -1,0 +1,29 @@
+"""Host logic of bench.py (CPU): committed traffic figures are used only while
+the sources they were measured on are unchanged, and scale by algorithmic bytes."""
+import json
+
+import bench
+
+
+def test_decode_traffic_follows_source_hash(tmp_path, monkeypatch):
+    path = tmp_path / "decode_traffic.json"
+    monkeypatch.setattr(bench, "DECODE_TRAFFIC_PATH", str(path))
+    good = bench.kernel_source_hash(("decode.cu", "sm100_ptx.cuh", "g3_internal.h"))
+    path.write_text(json.dumps({"bytes_per_algorithmic_byte": 1.25, "source_hash": good}))
+    assert bench.decode_traffic_per_launch(1000.0) == 1250.0
+    path.write_text(json.dumps({"bytes_per_algorithmic_byte": 1.25, "source_hash": "0" * 16}))
+    assert bench.decode_traffic_per_launch(1000.0) is None
+    path.write_text("not json")
+    assert bench.decode_traffic_per_launch(1000.0) is None
+
+
+def test_source_hash_depends_on_the_files():
+    a = bench.kernel_source_hash(("prefill.cu",))
+    b = bench.kernel_source_hash(("prefill.cu", "g3_internal.h"))
+    assert a != b and len(a) == 16
+    assert a == bench.kernel_source_hash(("prefill.cu",))
+
+
+def test_weak_scaling_rate_counts_every_rank():
+    # 2 ranks x 3 steps of 10 units in 6 ms (the slowest rank) = 10,000 units/s
+    assert bench.weak_scaling_rate(10.0, 3, 2, 6.0) == 10.0 * 3 * 2 / 6e-3
