@@ -123,7 +123,10 @@ bool make_bhsd_map(CUtensorMap* map, const void* base, int B, int H, int rows, i
 struct PrefillWs {
   size_t lo, hi, table, q_hat, k_hat, total;
 };
-bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w) {
+// The rotation table (cos, sin per token and frequency) is stored only for the
+// backward pass, which re-applies the rotation to the gradients; the forward
+// pass forms the angles in registers.
+bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w, bool with_table = false) {
   if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || D < 1) return false;
   const size_t rows = (size_t)B * S;
   size_t off = g3::kHeaderBytes;
@@ -132,7 +135,7 @@ bool prefill_ws(int B, int S, int Hq, int Hkv, int D, PrefillWs* w) {
   w->hi = off;
   off = align_up(off + rows * 4, 1024);
   w->table = off;
-  off = align_up(off + rows * (D / 2) * 8, 1024);
+  if (with_table) off = align_up(off + rows * (D / 2) * 8, 1024);
   w->q_hat = off;
   off = align_up(off + rows * Hq * D * 2, 1024);
   w->k_hat = off;
@@ -146,7 +149,7 @@ int chunk_hist(int start, g3_layer_kind kind, int window) {
   return kind == G3_LAYER_LOCAL ? std::min(start, window - 1) : start;
 }
 struct ChunkWs {
-  size_t lo, hi, table, q_hat, ctx_k, ctx_v, total;
+  size_t lo, hi, q_hat, ctx_k, ctx_v, total;
   int rows;  // K/V rows of the local context buffers (history + chunk)
 };
 bool chunk_ws(int B, int C, int Hq, int Hkv, int D, int start, g3_layer_kind kind, int window, ChunkWs* w) {
@@ -158,8 +161,6 @@ bool chunk_ws(int B, int C, int Hq, int Hkv, int D, int start, g3_layer_kind kin
   off = align_up(off + rows * 4, 1024);
   w->hi = off;
   off = align_up(off + rows * 4, 1024);
-  w->table = off;
-  off = align_up(off + rows * (D / 2) * 8, 1024);
   w->q_hat = off;
   off = align_up(off + rows * Hq * D * 2, 1024);
   w->rows = 0;
@@ -207,7 +208,7 @@ struct BwdWs {
   int S_pad, n_kvtiles;
 };
 bool bwd_ws(int B, int S, int Hq, int Hkv, int D, BwdWs* w) {
-  if (!prefill_ws(B, S, Hq, Hkv, D, &w->f)) return false;
+  if (!prefill_ws(B, S, Hq, Hkv, D, &w->f, /*with_table=*/true)) return false;
   w->n_kvtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
   w->S_pad = w->n_kvtiles * g3::kTileRows;
   size_t off = w->f.total;
