@@ -50,6 +50,25 @@ def peaks():
 DECODE_TRAFFIC_PATH = os.path.join(ROOT, "profiles", "decode_split_traffic.json")
 
 
+# The library's per-kernel trace brackets each launch with CUDA events; an event
+# between two kernels keeps the next launch from starting until the previous one
+# has drained (~5 us per kernel boundary, ~4 % of the 8K block step).  So the
+# timed loops carry the trace on every TRACE_EVERY-th step only (the first one
+# included), and a kernel's average duration comes from those steps' launches.
+TRACE_EVERY = 4
+
+
+def n_traced(steps: int) -> int:
+    """Timed steps that carry the trace: 0, TRACE_EVERY, 2*TRACE_EVERY, ..."""
+    return (steps + TRACE_EVERY - 1) // TRACE_EVERY
+
+
+def launches_in_timed_region(trace: dict, steps: int) -> int:
+    """All launches of the timed loop: the traced steps' launches per step times the steps."""
+    per_step = sum(v[0] for v in trace.values()) // max(n_traced(steps), 1)
+    return per_step * steps
+
+
 def kernel_source_hash(files=("prefill.cu", "sm100_ptx.cuh", "g3_internal.h")) -> str:
     """Hash of the sources a committed ncu traffic figure was taken on."""
     h = hashlib.sha256()
@@ -274,15 +293,15 @@ def run_gpu(args, rank, world, local_rank):
     g3.trace_collect()
     barrier()
     with sampler:
-        g3.trace_enable(True)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
+        for i in range(args.steps):
+            g3.trace_enable(i % TRACE_EVERY == 0)
             prefill_step()
+        g3.trace_enable(False)
         e1.record(stream)
         barrier()
-        g3.trace_enable(False)
     ms = e0.elapsed_time(e1)
     trace = g3.trace_collect()
     if g3.check_device_error(ws) != 0:
@@ -291,7 +310,7 @@ def run_gpu(args, rank, world, local_rank):
     value = weak_scaling_rate(block_flops, args.steps, world, ms_max) / 1e12
 
     n_attn, attn_ms = trace.get("prefill_attention", (0, 0.0))
-    achieved = block_flops * args.steps / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
+    achieved = block_flops * n_traced(args.steps) / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
     traffic = None
     try:
         with open(TRAFFIC_PATH) as f:
@@ -304,7 +323,9 @@ def run_gpu(args, rank, world, local_rank):
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
                 "kernel": "prefill_attention", "peak_kind": f"{pk_kind} dense bf16 burst",
-                "launches": n_attn, "avg_launch_ms": attn_ms / max(n_attn, 1)}
+                "launches": n_attn, "avg_launch_ms": attn_ms / max(n_attn, 1),
+                "traced_steps": n_traced(args.steps)}
+    # Launches and time of the traced steps (every TRACE_EVERY-th timed step).
     kernels = {k: {"launches": v[0], "ms": v[1], "share": v[1] / max(sum(x[1] for x in trace.values()), 1e-9)}
                for k, v in trace.items()}
 
@@ -455,15 +476,15 @@ def run_gpu(args, rank, world, local_rank):
         reps = max(args.steps // 2, 5)
         g3.trace_collect()
         barrier()
-        g3.trace_enable(True)
         e0b = torch.cuda.Event(enable_timing=True)
         e1b = torch.cuda.Event(enable_timing=True)
         e0b.record(stream)
-        for _ in range(reps):
+        for i in range(reps):
+            g3.trace_enable(i % TRACE_EVERY == 0)
             backward_block()
+        g3.trace_enable(False)
         e1b.record(stream)
         barrier()
-        g3.trace_enable(False)
         tr = g3.trace_collect()
         if g3.check_device_error(bws) != 0:
             raise RuntimeError("device error in the backward timing")
@@ -475,7 +496,7 @@ def run_gpu(args, rank, world, local_rank):
         ker = {}
         for name, mult in (("backward_dkdv", 2.0), ("backward_dq", 1.5)):
             n_k, m_k = tr.get(name, (0, 0.0))
-            tf = mult * block_flops * reps / (m_k * 1e-3) / 1e12 if m_k > 0 else None
+            tf = mult * block_flops * n_traced(reps) / (m_k * 1e-3) / 1e12 if m_k > 0 else None
             ker[name] = {"launches": n_k, "ms": m_k, "tflops_executed": tf,
                          "frac_of_measured_peak": tf / peak_tf if tf else None}
         for name in ("prefill_prologue", "backward_prep", "backward_norm_rope"):
@@ -591,7 +612,7 @@ def run_gpu(args, rank, world, local_rank):
         "shapes_1b": shapes_1b,
         "soft_tokens": soft,
         "backward": backward,
-        "gpu_launches": sum(v[0] for v in trace.values()),
+        "gpu_launches": launches_in_timed_region(trace, args.steps),
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
@@ -637,22 +658,22 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    g3.trace_enable(True)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        g3.trace_enable(i % TRACE_EVERY == 0)
         step()
+    g3.trace_enable(False)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    g3.trace_enable(False)
     if world > 1:
         torch.distributed.barrier()
     trace = g3.trace_collect()
     ms = max_over_ranks(e0.elapsed_time(e1), dev)
     gbs = weak_scaling_rate(step_bytes, args.steps, world, ms) / 1e9
     n_split, split_ms = trace.get("decode_split", (0, 0.0))
-    ach = step_bytes * args.steps / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
+    ach = step_bytes * n_traced(args.steps) / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
     del caches
     torch.cuda.empty_cache()
     return {
@@ -662,9 +683,10 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
         "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": (ach / pk["hbm_gbs"]) if ach else None,
                      "traffic": decode_traffic_per_launch(step_bytes / len(blk)), "kernel": "decode_split",
-                     "peak_kind": f"{pk_kind} copy bandwidth", "launches": n_split},
+                     "peak_kind": f"{pk_kind} copy bandwidth", "launches": n_split,
+                     "traced_steps": n_traced(args.steps)},
         "kernels": {k: {"launches": v[0], "ms": v[1]} for k, v in trace.items()},
-        "gpu_launches": sum(v[0] for v in trace.values()),
+        "gpu_launches": launches_in_timed_region(trace, args.steps),
     }
 
 

@@ -27,3 +27,17 @@ def test_source_hash_depends_on_the_files():
 def test_weak_scaling_rate_counts_every_rank():
     # 2 ranks x 3 steps of 10 units in 6 ms (the slowest rank) = 10,000 units/s
     assert bench.weak_scaling_rate(10.0, 3, 2, 6.0) == 10.0 * 3 * 2 / 6e-3
+
+
+def test_trace_sampling_counts():
+    # The trace rides on steps 0, TRACE_EVERY, 2*TRACE_EVERY, ... of the timed loop.
+    E = bench.TRACE_EVERY
+    assert bench.n_traced(1) == 1
+    assert bench.n_traced(E) == 1
+    assert bench.n_traced(E + 1) == 2
+    assert bench.n_traced(20) == len(range(0, 20, E))
+    # 12 launches per step on the traced steps scale to every timed step.
+    steps = 20
+    trace = {"prefill_prologue": (6 * bench.n_traced(steps), 1.0),
+             "prefill_attention": (6 * bench.n_traced(steps), 9.0)}
+    assert bench.launches_in_timed_region(trace, steps) == 12 * steps
