@@ -40,6 +40,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "func_attr.cuh"
 #include "g3_internal.h"
 #include "sm100_ptx.cuh"
 #include "tmem_wide.cuh"
@@ -712,13 +713,9 @@ static cudaError_t launch_dkdv_t(const BwdParams& p, const CUtensorMap& tq, cons
                                  const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
   using L = DkdvLayout<D>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};  // devices with the shared-memory limit raised
+  const cudaError_t e = ensure_dynamic_smem(bwd_dkdv_kernel<D>, L::kAlloc, configured);
+  if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)p.n_kvtiles * p.B * p.Hkv;
   bwd_dkdv_kernel<D><<<grid, kBwdThreads, L::kAlloc, st>>>(tq, tdo, tk, tv, p);
   return cudaGetLastError();
@@ -1025,12 +1022,9 @@ static cudaError_t launch_dq_t(const BwdParams& p, const CUtensorMap& tq, const 
                                const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
   using L = DqLayout<D>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};  // devices with the shared-memory limit raised
+  const cudaError_t e = ensure_dynamic_smem(bwd_dq_kernel<D>, L::kAlloc, configured);
+  if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hq;
   bwd_dq_kernel<D><<<grid, kBwdThreads, L::kAlloc, st>>>(tq, tdo, tk, tv, p);
   return cudaGetLastError();

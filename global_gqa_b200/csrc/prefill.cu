@@ -22,6 +22,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "func_attr.cuh"
 #include "g3_internal.h"
 #include "sm100_ptx.cuh"
 #include "tmem_wide.cuh"
@@ -433,13 +434,9 @@ static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, con
                                  const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t st) {
   using L = AttnLayout<D, HPC>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  static bool configured = false;  // the attribute belongs to the function; set it once
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(prefill_attention_kernel<D, HPC>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};  // devices with the shared-memory limit raised
+  const cudaError_t e = ensure_dynamic_smem(prefill_attention_kernel<D, HPC>, L::kAlloc, configured);
+  if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hkv * p.n_groups;
   prefill_attention_kernel<D, HPC><<<grid, AttnRoles<HPC>::kThreads, L::kAlloc, st>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
