@@ -136,8 +136,29 @@ def _ptr(t) -> Optional[int]:
 
 def _stream_ptr(stream, device) -> int:
     torch = _torch()
-    s = stream if stream is not None else torch.cuda.current_stream(device)
-    return s.cuda_stream
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if stream.device != device:
+        raise ValueError(f"stream belongs to {stream.device}; the call runs on {device}")
+    return stream.cuda_stream
+
+
+def _on_device(device, **tensors) -> None:
+    """Every tensor of one call lives on the GPU the call runs on (the library
+    launches on the current device, which the entry points set to it)."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}; every tensor of the call must be on {device}")
+
+
+def _ws(ws, nbytes: int, device, tag: str = "default"):
+    """The caller's workspace (checked) or the cached one, with its size in bytes."""
+    torch = _torch()
+    if ws is None:
+        ws = workspace(nbytes, device, tag)
+    elif not isinstance(ws, torch.Tensor) or ws.device != device or not ws.is_contiguous():
+        raise ValueError(f"ws must be a contiguous tensor on {device}")
+    return ws, ws.numel() * ws.element_size()
 
 
 def _req(t, name, dtype, shape=None):
@@ -181,19 +202,25 @@ def prefill(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, window: int, 
             image_spans = None
     if out is None:
         out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, S, Hq, D))
     lse = torch.empty(B, Hq, S, dtype=torch.float32, device=q.device) if return_lse else None
     cap = 0
     if k_cache is not None:
         _req(k_cache, "k_cache", torch.bfloat16)
+        if k_cache.dim() != 4 or k_cache.shape[0] != B or k_cache.shape[1] != Hkv or k_cache.shape[3] != D:
+            raise ValueError("k_cache must be [B, Hkv, capacity, D]")
         _req(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
         cap = int(k_cache.shape[2])
-    need = prefill_workspace_size(B, S, Hq, Hkv, D)
-    wsb = ws if ws is not None else workspace(need, q.device)
-    st = lib().g3attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
-                              int(layer_kind), int(window), float(rope_base), float(interp_factor),
-                              _ptr(image_spans), n_spans, B, S, Hq, Hkv, D, _ptr(out), _ptr(lse),
-                              _ptr(k_cache), _ptr(v_cache), cap, wsb.data_ptr(), wsb.numel(),
-                              _stream_ptr(stream, q.device))
+    dev = q.device
+    _on_device(dev, k=k, v=v, q_gamma=q_gamma, k_gamma=k_gamma, positions=positions, image_spans=image_spans,
+               out=out, k_cache=k_cache, v_cache=v_cache)
+    wsb, ws_bytes = _ws(ws, prefill_workspace_size(B, S, Hq, Hkv, D), dev)
+    with torch.cuda.device(dev):
+        st = lib().g3attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
+                                  int(layer_kind), int(window), float(rope_base), float(interp_factor),
+                                  _ptr(image_spans), n_spans, B, S, Hq, Hkv, D, _ptr(out), _ptr(lse),
+                                  _ptr(k_cache), _ptr(v_cache), cap, wsb.data_ptr(), ws_bytes,
+                                  _stream_ptr(stream, dev))
     _check(st, "g3attn_prefill")
     return (out, lse) if return_lse else out
 
@@ -237,14 +264,17 @@ def prefill_backward(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, wind
     _req(g["dv"], "dv", torch.bfloat16, (B, S, Hkv, D))
     _req(g["dq_gamma"], "dq_gamma", torch.float32, (D,))
     _req(g["dk_gamma"], "dk_gamma", torch.float32, (D,))
-    need = prefill_backward_workspace_size(B, S, Hq, Hkv, D)
-    wsb = ws if ws is not None else workspace(need, q.device, tag="backward")
-    st = lib().g3attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
-                                       int(layer_kind), int(window), float(rope_base), float(interp_factor),
-                                       _ptr(image_spans), n_spans, B, S, Hq, Hkv, D, _ptr(out), _ptr(lse),
-                                       _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
-                                       _ptr(g["dq_gamma"]), _ptr(g["dk_gamma"]), wsb.data_ptr(), wsb.numel(),
-                                       _stream_ptr(stream, q.device))
+    dev = q.device
+    _on_device(dev, k=k, v=v, q_gamma=q_gamma, k_gamma=k_gamma, positions=positions, image_spans=image_spans,
+               out=out, lse=lse, dout=dout, **g)
+    wsb, ws_bytes = _ws(ws, prefill_backward_workspace_size(B, S, Hq, Hkv, D), dev, tag="backward")
+    with torch.cuda.device(dev):
+        st = lib().g3attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma),
+                                           _ptr(positions), int(layer_kind), int(window), float(rope_base),
+                                           float(interp_factor), _ptr(image_spans), n_spans, B, S, Hq, Hkv, D,
+                                           _ptr(out), _ptr(lse), _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]),
+                                           _ptr(g["dv"]), _ptr(g["dq_gamma"]), _ptr(g["dk_gamma"]),
+                                           wsb.data_ptr(), ws_bytes, _stream_ptr(stream, dev))
     _check(st, "g3attn_prefill_backward")
     return g
 
@@ -268,13 +298,16 @@ def decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, seq_lens, max_se
     _req(seq_lens, "seq_lens", torch.int32, (B,))
     if out is None:
         out = torch.empty_like(q)
-    need = decode_workspace_size(B, Hq, Hkv, D, max_seq_len)
-    wsb = ws if ws is not None else workspace(need, q.device)
-    st = lib().g3attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_gamma), _ptr(k_gamma),
-                             _ptr(k_cache), _ptr(v_cache), cap, _ptr(seq_lens), int(max_seq_len),
-                             int(layer_kind), int(window), float(rope_base), float(interp_factor),
-                             B, Hq, Hkv, D, _ptr(out), wsb.data_ptr(), wsb.numel(),
-                             _stream_ptr(stream, q.device))
+    _req(out, "out", torch.bfloat16, (B, Hq, D))
+    dev = q.device
+    _on_device(dev, k_new=k_new, v_new=v_new, q_gamma=q_gamma, k_gamma=k_gamma, k_cache=k_cache,
+               v_cache=v_cache, seq_lens=seq_lens, out=out)
+    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, max_seq_len), dev)
+    with torch.cuda.device(dev):
+        st = lib().g3attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_gamma), _ptr(k_gamma),
+                                 _ptr(k_cache), _ptr(v_cache), cap, _ptr(seq_lens), int(max_seq_len),
+                                 int(layer_kind), int(window), float(rope_base), float(interp_factor),
+                                 B, Hq, Hkv, D, _ptr(out), wsb.data_ptr(), ws_bytes, _stream_ptr(stream, dev))
     _check(st, "g3attn_decode")
     return out
 
@@ -285,7 +318,10 @@ def check_device_error(ws=None, device=None, stream=None) -> int:
     if ws is None:
         dev = torch.device(device if device is not None else "cuda")
         ws = workspace(256, dev)
-    return int(lib().g3attn_check_device_error(ws.data_ptr(), _stream_ptr(stream, ws.device)))
+    if not isinstance(ws, torch.Tensor) or ws.device.type != "cuda":
+        raise ValueError("ws must be a CUDA tensor")
+    with torch.cuda.device(ws.device):
+        return int(lib().g3attn_check_device_error(ws.data_ptr(), _stream_ptr(stream, ws.device)))
 
 
 def trace_enable(on: bool = True) -> None:
@@ -331,16 +367,21 @@ def prefill_chunk(q, k, v, q_gamma, k_gamma, positions, k_cache, v_cache, start:
             image_spans = None
     if out is None:
         out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, (B, C, Hq, D))
     lse = torch.empty(B, Hq, C, dtype=torch.float32, device=q.device) if return_lse else None
     need = prefill_chunk_workspace_size(B, C, Hq, Hkv, D, start, layer_kind, window)
     if need == 0:
         raise ValueError("invalid sizes for prefill_chunk")
-    wsb = ws if ws is not None else workspace(need, q.device)
-    st = lib().g3attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
-                                    _ptr(k_cache), _ptr(v_cache), cap, int(start), int(layer_kind), int(window),
-                                    float(rope_base), float(interp_factor), _ptr(image_spans), n_spans, B, C, Hq,
-                                    Hkv, D, _ptr(out), _ptr(lse), wsb.data_ptr(), wsb.numel(),
-                                    _stream_ptr(stream, q.device))
+    dev = q.device
+    _on_device(dev, k=k, v=v, q_gamma=q_gamma, k_gamma=k_gamma, positions=positions, k_cache=k_cache,
+               v_cache=v_cache, image_spans=image_spans, out=out)
+    wsb, ws_bytes = _ws(ws, need, dev)
+    with torch.cuda.device(dev):
+        st = lib().g3attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
+                                        _ptr(k_cache), _ptr(v_cache), cap, int(start), int(layer_kind),
+                                        int(window), float(rope_base), float(interp_factor), _ptr(image_spans),
+                                        n_spans, B, C, Hq, Hkv, D, _ptr(out), _ptr(lse), wsb.data_ptr(),
+                                        ws_bytes, _stream_ptr(stream, dev))
     _check(st, "g3attn_prefill_chunk")
     return (out, lse) if return_lse else out
 
@@ -360,7 +401,10 @@ def soft_tokens(patches, gamma, grid_h: int, grid_w: int, pool: int = 4, *, out=
     if out is None:
         out = torch.empty(B, n_out, F, dtype=torch.bfloat16, device=patches.device)
     _req(out, "out", torch.bfloat16, (B, n_out, F))
-    st = lib().g3attn_soft_tokens(_ptr(patches), _ptr(gamma), B, grid_h, grid_w, F, pool, _ptr(out),
-                                  _stream_ptr(stream, patches.device))
+    dev = patches.device
+    _on_device(dev, gamma=gamma, out=out)
+    with torch.cuda.device(dev):
+        st = lib().g3attn_soft_tokens(_ptr(patches), _ptr(gamma), B, grid_h, grid_w, F, pool, _ptr(out),
+                                      _stream_ptr(stream, dev))
     _check(st, "g3attn_soft_tokens")
     return out
