@@ -735,7 +735,9 @@ def main():
         import datetime
         import torch
         torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        # Every rank runs the same work between collectives, so a rank that
+        # stalls or dies shows as a collective timing out well within this.
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                              device_id=torch.device("cuda", local_rank))
     line = run_gpu(args, rank, world, local_rank)
     if rank == 0 and world == 1:
