@@ -66,7 +66,12 @@ def _i64(x) -> np.ndarray:
 
 # ---------------------------------------------------------------- step 1 --
 def qk_rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float = EPS) -> np.ndarray:
-    """x / sqrt(mean_d x_d^2 + eps) * gamma over the last axis (head_dim)."""
+    """x / sqrt(mean_d x_d^2 + eps) * gamma over the last axis (head_dim).
+
+    Gemma 3 Technical Report, section 2 "Model Architecture" (QK-norm); eps and
+    the normalised axis from the q_norm/k_norm lines printed on "Gemma
+    explained: what's new in Gemma 3".
+    """
     x = _f64(x)
     g = _f64(gamma)
     ms = np.mean(x * x, axis=-1, keepdims=True)
@@ -75,7 +80,8 @@ def qk_rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float = EPS) -> np.ndarray
 
 # ---------------------------------------------------------------- step 2 --
 def inv_frequencies(D: int, base: float) -> np.ndarray:
-    """base^(-2d/D) for d = 0 .. D/2-1."""
+    """base^(-2d/D) for d = 0 .. D/2-1 (Technical Report, section 2 "Long context":
+    base 10k on local layers, 1M on global layers)."""
     d = np.arange(D // 2, dtype=np.float64)
     return np.power(float(base), -2.0 * d / D)
 
@@ -85,6 +91,8 @@ def rope(x: np.ndarray, pos: np.ndarray, base: float, interp: float = 1.0) -> np
 
     Pair (x_d, x_{d+D/2}) becomes (x_d cos t - x_{d+D/2} sin t,
     x_d sin t + x_{d+D/2} cos t) with t = (pos / interp) * base^(-2d/D).
+    Technical Report, section 2 "Long context" (bases; linear interpolation
+    "similar to Chen et al. (2023)"); the half-split pairing is a reading.
     """
     x = _f64(x)
     p = _f64(pos) / float(interp)
@@ -100,7 +108,9 @@ def rope(x: np.ndarray, pos: np.ndarray, base: float, interp: float = 1.0) -> np
 
 # ---------------------------------------------------------------- step 3 --
 def span_ids(S: int, spans_b: Optional[np.ndarray]) -> np.ndarray:
-    """Per token: index of the image span [start, end) holding it, else -1."""
+    """Per token: index of the image span [start, end) holding it, else -1
+    ("Gemma explained", section "Vision encoder and processing": 256 soft
+    tokens per image)."""
     sid = np.full(S, -1, dtype=np.int64)
     if spans_b is None:
         return sid
@@ -110,7 +120,13 @@ def span_ids(S: int, spans_b: Optional[np.ndarray]) -> np.ndarray:
 
 
 def allowed(i, j, kind: int, window: int, sid: np.ndarray) -> np.ndarray:
-    """The visibility predicate, vectorised over broadcastable i and j."""
+    """The visibility predicate, vectorised over broadcastable i and j.
+
+    Causal window of W keys on local layers, all earlier keys on global ones
+    (Technical Report, section 1 Introduction and section 2 "5:1 interleaving
+    of local/global layers"), joined with bidirectional attention inside one
+    image ("Gemma explained", section "Vision encoder and processing").
+    """
     i = np.asarray(i, dtype=np.int64)
     j = np.asarray(j, dtype=np.int64)
     causal = j <= i
@@ -121,11 +137,13 @@ def allowed(i, j, kind: int, window: int, sid: np.ndarray) -> np.ndarray:
 
 
 def allowed_row(i: int, S: int, kind: int, window: int, sid: np.ndarray) -> np.ndarray:
+    """Visibility of every key j < S from query i (`allowed` on one row)."""
     return allowed(np.int64(i), np.arange(S, dtype=np.int64), kind, window, sid)
 
 
 def unmasked_pairs(S: int, kind: int, window: int, spans_b=None) -> int:
-    """Number of visible (i, j) pairs of one sequence, by enumeration."""
+    """Number of visible (i, j) pairs of one sequence, by enumeration of
+    `allowed` (the predicate of step 3 above)."""
     sid = span_ids(S, spans_b)
     total = 0
     for i in range(S):
@@ -179,7 +197,9 @@ def prefill_rows(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_base, 
     q [B,S,Hq,D], k/v [B,S,Hkv,D] raw (pre-norm, pre-RoPE); positions [B,S];
     spans [B,n,2] half-open or None; rows: 1-D list of row indices (all rows
     if None), the same for every sequence.
-    Returns (out [B, R, Hq, D], lse [B, Hq, R]) in float64.
+    Returns (out [B, R, Hq, D], lse [B, Hq, R]) in float64.  Steps 1-5 of the
+    module docstring: GQA head mapping from the Technical Report, section 2;
+    softmax with scale 1/sqrt(D) over each row's visible set.
     """
     B, S, Hq, D = q.shape
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
@@ -207,7 +227,8 @@ def prefill_rows(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_base, 
 
 
 def prefill(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_base, interp, spans=None):
-    """All rows: out [B,S,Hq,D] and lse [B,Hq,S] (float64)."""
+    """All rows: out [B,S,Hq,D] and lse [B,Hq,S] (float64); steps 1-5 of the
+    module docstring (Technical Report, section 2; "Gemma explained")."""
     return prefill_rows(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_base,
                         interp, spans, rows=None)
 
@@ -217,7 +238,8 @@ def prefill_bruteforce(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_
     """Second formulation: the full S x S score matrix per head, masked.
 
     Loops over every (batch, query head) and builds the whole mask with the
-    predicate; meant for tiny inputs only.
+    predicate; meant for tiny inputs only.  Same definition and sources as
+    `prefill`.
     """
     qh, kh, vf = _prepare(q, k, v, q_gamma, k_gamma, positions, rope_base, interp)
     B, S, Hq, D = qh.shape
@@ -254,6 +276,9 @@ def decode(q, k_new, v_new, q_gamma, k_gamma, seq_lens, k_hist, v_hist, hist_sta
     older than hist_start[b] must be invisible from row L-1.
 
     Returns out [B,Hq,D] and the new token's rotated key k_hat [B,Hkv,D].
+    The 1024-slot ring of local layers follows from the window (Technical
+    Report, section 2 "5:1 interleaving": only global layers keep the long
+    context's KV cache).
     """
     qf = _f64(q)
     B, Hq, D = qf.shape

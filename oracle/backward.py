@@ -48,7 +48,11 @@ __all__ = ["rope_backward", "rmsnorm_backward", "attention_backward", "prefill_b
 
 # --------------------------------------------------------------- step 2' --
 def rope_backward(g: np.ndarray, pos: np.ndarray, base: float, interp: float = 1.0) -> np.ndarray:
-    """Gradient through the rotation: g [..., T, H, D] at positions pos [..., T]."""
+    """Gradient through the rotation: g [..., T, H, D] at positions pos [..., T].
+
+    Step 2' of the module docstring: the inverse of the rotation that
+    `oracle.attention.rope` applies (Technical Report, section 2 "Long context").
+    """
     g = _f64(g)
     p = _f64(pos) / float(interp)
     D = g.shape[-1]
@@ -66,6 +70,8 @@ def rmsnorm_backward(x: np.ndarray, gamma: np.ndarray, g: np.ndarray, eps: float
     """Gradient of y = x / sqrt(mean(x^2) + eps) * gamma over the last axis.
 
     Returns (dx with the shape of x, dgamma [D] summed over all other axes).
+    Step 1' of the module docstring: the chain rule through the QK-norm of the
+    Technical Report, section 2 "Model Architecture".
     """
     x = _f64(x)
     gm = _f64(gamma)
@@ -86,7 +92,10 @@ def attention_backward(qh, kh, v, dout, kind: int, window: int, sid: np.ndarray,
     qh [S, Hq, D], kh / v [S, Hkv, D] (normalised and rotated q and k, raw v),
     dout [S, Hq, D].  Only the kv heads in `kv_heads` (all if None) and their
     query heads are computed; the other heads of the results are NaN.
-    Returns dqh [S, Hq, D], dkh [S, Hkv, D], dv [S, Hkv, D].
+    Returns dqh [S, Hq, D], dkh [S, Hkv, D], dv [S, Hkv, D].  Steps 5', 4' and
+    3' of the module docstring, over the forward's visible sets (Technical
+    Report, section 2; "Gemma explained", section "Vision encoder and
+    processing").
     """
     qh, kh, v, dout = _f64(qh), _f64(kh), _f64(v), _f64(dout)
     S, Hq, D = qh.shape
@@ -126,7 +135,9 @@ def attention_backward(qh, kh, v, dout, kind: int, window: int, sid: np.ndarray,
 # ------------------------------------------------------------ whole call --
 def prefill_backward(q, k, v, q_gamma, k_gamma, positions, kind, window, rope_base, interp, dout,
                      spans=None, kv_heads: Optional[Sequence[int]] = None, row_group: int = 256):
-    """Gradients of sum(out * dout) for one prefill call of the block.
+    """Gradients of sum(out * dout) for one prefill call of the block (steps 5'
+    to 1' of the module docstring; the training that needs them: Technical
+    Report, sections 2.2 "Pre-training" and 2.3 "Quantization Aware Training").
 
     q [B,S,Hq,D], k/v [B,S,Hkv,D] raw (pre-norm, pre-RoPE), gammas [D],
     positions [B,S], spans [B,n,2] or None, dout [B,S,Hq,D].

@@ -35,6 +35,9 @@ def soft_tokens(patches, gamma, grid_h: int, grid_w: int, pool: int = 4):
     Step 1: average each pool x pool block of the patch grid (no padding).
     Step 2: RMS-normalise every pooled vector over its F features (eps 1e-6)
             and multiply by gamma.
+    The projector's printed modules and the 256 tokens per image: "Gemma
+    explained: what's new in Gemma 3", the 27B model's printout and section
+    "Vision encoder and processing".
     """
     x = np.asarray(patches, dtype=np.float64)
     g = np.asarray(gamma, dtype=np.float64)
