@@ -4,12 +4,14 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/g3attn.h"
@@ -34,22 +36,29 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ------------------------------------------------------------------ tracing
+// Events belong to the device that was current when they were created, and
+// may only be recorded on that device's streams, so both the pending entries
+// and the pool of reusable events carry their device.
 struct TraceEntry {
   std::string name;
+  int device;
   cudaEvent_t start, stop;
 };
 struct TraceState {
   std::mutex mu;
-  bool enabled = false;
+  std::atomic<bool> enabled{false};
   std::vector<TraceEntry> pending;
-  std::vector<cudaEvent_t> pool;
+  std::vector<std::pair<int, cudaEvent_t>> pool;  // (device, event)
 } g_trace;
 
-cudaEvent_t trace_event() {
-  if (!g_trace.pool.empty()) {
-    cudaEvent_t e = g_trace.pool.back();
-    g_trace.pool.pop_back();
-    return e;
+// An event of device `dev` (the current device); the caller holds g_trace.mu.
+cudaEvent_t trace_event(int dev) {
+  for (size_t i = g_trace.pool.size(); i-- > 0;) {
+    if (g_trace.pool[i].first == dev) {
+      const cudaEvent_t e = g_trace.pool[i].second;
+      g_trace.pool.erase(g_trace.pool.begin() + (std::ptrdiff_t)i);
+      return e;
+    }
   }
   cudaEvent_t e = nullptr;
   cudaEventCreate(&e);
@@ -59,9 +68,11 @@ cudaEvent_t trace_event() {
 // Runs `launch` bracketed by trace events when tracing is on.
 template <class F>
 cudaError_t traced(const char* name, cudaStream_t st, F&& launch) {
-  if (!g_trace.enabled) return launch();
+  if (!g_trace.enabled.load(std::memory_order_relaxed)) return launch();
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return launch();
   std::lock_guard<std::mutex> lk(g_trace.mu);
-  TraceEntry e{name, trace_event(), trace_event()};
+  TraceEntry e{name, dev, trace_event(dev), trace_event(dev)};
   cudaEventRecord(e.start, st);
   cudaError_t r = launch();
   cudaEventRecord(e.stop, st);
@@ -793,7 +804,7 @@ g3_status g3attn_check_device_error(void* workspace, void* stream) {
 
 g3_status g3attn_trace_enable(int enable) {
   std::lock_guard<std::mutex> lk(g_trace.mu);
-  g_trace.enabled = enable != 0;
+  g_trace.enabled.store(enable != 0, std::memory_order_relaxed);
   return G3_OK;
 }
 
@@ -814,8 +825,8 @@ int32_t g3attn_trace_collect(g3_kernel_trace* out, int32_t max_entries) {
     }
     slot->launches += 1;
     slot->total_ms += ms;
-    g_trace.pool.push_back(t.start);
-    g_trace.pool.push_back(t.stop);
+    g_trace.pool.emplace_back(t.device, t.start);
+    g_trace.pool.emplace_back(t.device, t.stop);
   }
   g_trace.pending.clear();
   const int n = (int)agg.size() < max_entries ? (int)agg.size() : max_entries;
