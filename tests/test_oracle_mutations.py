@@ -80,7 +80,44 @@ def _attend_factory(gqa_mod=False, no_scale=False):
     return attend
 
 
+def _decode_factory(pos_shift=0, gqa_mod=False, value_is_key=False, no_scale=False):
+    """Copy of the oracle's decode step with one planted mistake."""
+    def decode(q, k_new, v_new, q_gamma, k_gamma, seq_lens, k_hist, v_hist, hist_start,
+               kind, window, rope_base, interp):
+        qf = O._f64(q)
+        B, Hq, D = qf.shape
+        L = O._i64(seq_lens)
+        out = np.empty((B, Hq, D))
+        k_hat = np.empty((B, O._f64(k_new).shape[1], D))
+        for b in range(B):
+            Lb = int(L[b])
+            pos = np.array([Lb - 1 + pos_shift], dtype=np.float64)
+            qh = O.rope(O.qk_rmsnorm(qf[b][None], q_gamma), pos, rope_base, interp)[0]
+            kn = O.rope(O.qk_rmsnorm(O._f64(k_new)[b][None], k_gamma), pos, rope_base, interp)[0]
+            k_hat[b] = kn
+            t0 = int(hist_start[b])
+            keys = np.concatenate([O._f64(k_hist[b]), kn[None]], axis=0)
+            newv = kn if value_is_key else O._f64(v_new)[b]
+            vals = np.concatenate([O._f64(v_hist[b]), newv[None]], axis=0)
+            vis = O.allowed(np.int64(Lb - 1), np.arange(t0, Lb), kind, window, O.span_ids(Lb, None))
+            Hkv = keys.shape[1]
+            for h in range(Hq):
+                kv = (h % Hkv) if gqa_mod else (h // (Hq // Hkv))
+                sc = keys[:, kv, :] @ qh[h]
+                if not no_scale:
+                    sc = sc / math.sqrt(D)
+                sc = np.where(vis, sc, -np.inf)
+                m = sc.max(); pr = np.exp(sc - m)
+                out[b, h] = pr @ vals[:, kv, :] / pr.sum()
+        return out, k_hat
+    return decode
+
+
 MUTANTS = {
+    "decode_position_off_by_one": ("decode", _decode_factory(pos_shift=1)),
+    "decode_gqa_head_modulo": ("decode", _decode_factory(gqa_mod=True)),
+    "decode_new_value_is_its_key": ("decode", _decode_factory(value_is_key=True)),
+    "decode_no_softmax_scale": ("decode", _decode_factory(no_scale=True)),
     "norm_drops_eps": ("qk_rmsnorm", _norm_no_eps),
     "norm_drops_gamma": ("qk_rmsnorm", _norm_no_gamma),
     "rope_reversed_sign": ("rope", _rope_factory(sign=-1.0)),
@@ -94,6 +131,18 @@ MUTANTS = {
     "gqa_head_modulo": ("_attend_rows", _attend_factory(gqa_mod=True)),
     "no_softmax_scale": ("_attend_rows", _attend_factory(no_scale=True)),
 }
+
+
+def test_unmutated_decode_copy_matches():
+    """The copy of decode used for mutants agrees with the oracle when unmutated."""
+    for kind, W, L in [(O.LOCAL, 7, 20), (O.GLOBAL, 1, 13)]:
+        q, k, v, qg, kg, kh, full, base, interp = P._decode_case(kind, W, L, 5)
+        args = (q[:, L - 1], k[:, L - 1], v[:, L - 1], qg, kg, [L], [kh[0, :L - 1]], [v[0, :L - 1]], [0],
+                kind, W, base, interp)
+        a, ka = O.decode(*args)
+        b, kb = _decode_factory()(*args)
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(ka, kb, rtol=1e-12, atol=1e-13)
 
 
 def test_unmutated_attend_matches():
