@@ -15,7 +15,8 @@ import test_oracle_pins as P
 
 def _norm_no_eps(x, gamma, eps=O.EPS):
     x = O._f64(x); g = O._f64(gamma)
-    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) * g
+    with np.errstate(invalid="ignore", divide="ignore"):  # a zero row gives NaN: what a pin catches
+        return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) * g
 
 
 def _norm_no_gamma(x, gamma, eps=O.EPS):
