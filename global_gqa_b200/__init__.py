@@ -119,13 +119,26 @@ def _torch():
 _workspaces = {}
 
 
-def workspace(nbytes: int, device, tag: str = "default"):
-    """A cached uint8 device buffer of at least nbytes (256-byte aligned)."""
+def workspace(nbytes: int, device, tag: str = "default", stream=None):
+    """A cached uint8 device buffer of at least nbytes (256-byte aligned).
+
+    One buffer per (device, tag, stream): calls on one stream run in order and
+    may share it, calls on different streams may overlap and must not (stream
+    None is the device's current stream, as in the calls).
+    """
     torch = _torch()
-    key = (str(device), tag)
+    device = torch.device(device)
+    if device.index is None:  # "cuda" means the current device: name it as tensors do
+        device = torch.device("cuda", torch.cuda.current_device())
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (str(device), tag, int(s.cuda_stream))
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        # Allocated on the stream that uses it, so that when a larger buffer
+        # replaces it, torch reuses the old memory only after that stream's
+        # earlier calls have finished with it.
+        with torch.cuda.stream(s):
+            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
         _workspaces[key] = buf
     return buf
 
@@ -151,11 +164,11 @@ def _on_device(device, **tensors) -> None:
             raise ValueError(f"{name} is on {t.device}; every tensor of the call must be on {device}")
 
 
-def _ws(ws, nbytes: int, device, tag: str = "default"):
-    """The caller's workspace (checked) or the cached one, with its size in bytes."""
+def _ws(ws, nbytes: int, device, tag: str = "default", stream=None):
+    """The caller's workspace (checked) or the stream's cached one, with its size in bytes."""
     torch = _torch()
     if ws is None:
-        ws = workspace(nbytes, device, tag)
+        ws = workspace(nbytes, device, tag, stream)
     elif not isinstance(ws, torch.Tensor) or ws.device != device or not ws.is_contiguous():
         raise ValueError(f"ws must be a contiguous tensor on {device}")
     return ws, ws.numel() * ws.element_size()
@@ -214,7 +227,7 @@ def prefill(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, window: int, 
     dev = q.device
     _on_device(dev, k=k, v=v, q_gamma=q_gamma, k_gamma=k_gamma, positions=positions, image_spans=image_spans,
                out=out, k_cache=k_cache, v_cache=v_cache)
-    wsb, ws_bytes = _ws(ws, prefill_workspace_size(B, S, Hq, Hkv, D), dev)
+    wsb, ws_bytes = _ws(ws, prefill_workspace_size(B, S, Hq, Hkv, D), dev, stream=stream)
     with torch.cuda.device(dev):
         st = lib().g3attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
                                   int(layer_kind), int(window), float(rope_base), float(interp_factor),
@@ -267,7 +280,8 @@ def prefill_backward(q, k, v, q_gamma, k_gamma, positions, layer_kind: int, wind
     dev = q.device
     _on_device(dev, k=k, v=v, q_gamma=q_gamma, k_gamma=k_gamma, positions=positions, image_spans=image_spans,
                out=out, lse=lse, dout=dout, **g)
-    wsb, ws_bytes = _ws(ws, prefill_backward_workspace_size(B, S, Hq, Hkv, D), dev, tag="backward")
+    wsb, ws_bytes = _ws(ws, prefill_backward_workspace_size(B, S, Hq, Hkv, D), dev, tag="backward",
+                        stream=stream)
     with torch.cuda.device(dev):
         st = lib().g3attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma),
                                            _ptr(positions), int(layer_kind), int(window), float(rope_base),
@@ -302,7 +316,7 @@ def decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, seq_lens, max_se
     dev = q.device
     _on_device(dev, k_new=k_new, v_new=v_new, q_gamma=q_gamma, k_gamma=k_gamma, k_cache=k_cache,
                v_cache=v_cache, seq_lens=seq_lens, out=out)
-    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, max_seq_len), dev)
+    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, max_seq_len), dev, stream=stream)
     with torch.cuda.device(dev):
         st = lib().g3attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_gamma), _ptr(k_gamma),
                                  _ptr(k_cache), _ptr(v_cache), cap, _ptr(seq_lens), int(max_seq_len),
@@ -317,7 +331,7 @@ def check_device_error(ws=None, device=None, stream=None) -> int:
     torch = _torch()
     if ws is None:
         dev = torch.device(device if device is not None else "cuda")
-        ws = workspace(256, dev)
+        ws = workspace(256, dev, stream=stream)
     if not isinstance(ws, torch.Tensor) or ws.device.type != "cuda":
         raise ValueError("ws must be a CUDA tensor")
     with torch.cuda.device(ws.device):
@@ -375,7 +389,7 @@ def prefill_chunk(q, k, v, q_gamma, k_gamma, positions, k_cache, v_cache, start:
     dev = q.device
     _on_device(dev, k=k, v=v, q_gamma=q_gamma, k_gamma=k_gamma, positions=positions, k_cache=k_cache,
                v_cache=v_cache, image_spans=image_spans, out=out)
-    wsb, ws_bytes = _ws(ws, need, dev)
+    wsb, ws_bytes = _ws(ws, need, dev, stream=stream)
     with torch.cuda.device(dev):
         st = lib().g3attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_gamma), _ptr(k_gamma), _ptr(positions),
                                         _ptr(k_cache), _ptr(v_cache), cap, int(start), int(layer_kind),

@@ -32,3 +32,48 @@ def test_stream_of_another_device_is_rejected():
         cuda_stream = 0
     with pytest.raises(ValueError, match="stream belongs to"):
         g3._stream_ptr(FakeStream(), torch.device("cuda", 0))
+
+
+class _FakeStream:
+    def __init__(self, handle):
+        self.cuda_stream = handle
+
+
+class _FakeTorch:
+    """The few torch calls the workspace cache makes, without a GPU."""
+    uint8 = torch.uint8
+    device = torch.device
+
+    class cuda:  # noqa: N801 (mirrors torch.cuda)
+        current = _FakeStream(0)
+
+        @staticmethod
+        def current_device():
+            return 0
+
+        @staticmethod
+        def current_stream(device=None):
+            return _FakeTorch.cuda.current
+
+        @staticmethod
+        def stream(s):
+            import contextlib
+            return contextlib.nullcontext()
+
+    @staticmethod
+    def empty(n, dtype, device):
+        return torch.empty(n, dtype=dtype)  # stands in for the device buffer
+
+
+def test_workspace_cache_is_per_device_and_stream(monkeypatch):
+    monkeypatch.setattr(g3, "_torch", lambda: _FakeTorch)
+    monkeypatch.setattr(g3, "_workspaces", {})
+    a = g3.workspace(512, torch.device("cuda", 0))
+    assert g3.workspace(256, "cuda") is a                       # "cuda" names the current device
+    assert g3.workspace(512, "cuda:0", stream=_FakeStream(0)) is a  # the current stream, named
+    b = g3.workspace(512, "cuda:0", stream=_FakeStream(7))
+    assert b is not a                                            # another stream, another buffer
+    assert g3.workspace(512, "cuda:0", tag="backward") is not a  # another tag, another buffer
+    c = g3.workspace(4096, "cuda:0")
+    assert c is not a and c.numel() >= 4096                      # grown on demand
+    assert g3.workspace(100, "cuda:0") is c
