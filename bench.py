@@ -30,7 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import inputs  # noqa: E402
-from global_gqa_b200 import metrics  # noqa: E402
+from global_gqa_b200 import metrics, shard  # noqa: E402
 
 METRIC = "prefill attn TFLOP/s (unmasked FLOPs, 5:1 block) & decode KV GB/s, 1 B200"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -139,6 +139,15 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def block_config(cfg, world: int, block_flops: float) -> dict:
+    """The `config` object of a block-prefill line; both arms print this one."""
+    return {"workload": cfg.name, "batch": cfg.B, "seq_len": cfg.S, "q_heads": cfg.Hq, "kv_heads": cfg.Hkv,
+            "head_dim": cfg.D, "block": "5 local (W=1024, base 1e4) + 1 global (base 1e6, interp 8)",
+            "unmasked_flops_per_step": block_flops,
+            "l2": "inputs larger than L2: each layer reads 128 MiB of q/k/v and writes 64 MiB",
+            "parallelism": f"independent replicas x{world}"}
 
 
 # ------------------------------------------------------- multi-rank helpers
@@ -264,10 +273,12 @@ def run_gpu(args, rank, world, local_rank):
     cfg = inputs.BLOCK_8K
     blk = cfg.block()
 
-    # ---- prefill block inputs, resident in HBM (one set per layer)
+    # ---- prefill block inputs, resident in HBM (one set per layer); under
+    # torchrun every rank takes a sequence of its own (seeded by rank)
     layers = []
     for li, L in enumerate(blk):
-        x = inputs.config_layer_inputs(cfg, li)
+        x = inputs.prefill_layer_inputs(cfg.B, cfg.S, cfg.Hq, cfg.Hkv, cfg.D, seed=cfg.seed + rank, layer=li,
+                                        n_spans=cfg.n_spans)
         xd = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
         xd["out"] = torch.empty_like(xd["q"])
         layers.append((L, xd))
@@ -593,18 +604,19 @@ def run_gpu(args, rank, world, local_rank):
     # ---- decode block step on the 64 x (4K..128K) workload
     decode = None
     if not args.no_decode:
-        decode = run_decode(args, dev, stream, world, pk, pk_kind)
+        decode = run_decode(args, dev, stream, rank, world, pk, pk_kind)
+
+    # ---- mixed text+image 2 x 32K block and 128K block
+    long_blocks = None
+    if args.extras:
+        long_blocks = run_long_blocks(args, dev, stream, rank, world, pk, pk_kind)
 
     clocks = sampler.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": cfg.name, "batch": cfg.B, "seq_len": cfg.S, "q_heads": cfg.Hq, "kv_heads": cfg.Hkv,
-                   "head_dim": cfg.D, "block": "5 local (W=1024, base 1e4) + 1 global (base 1e6, interp 8)",
-                   "unmasked_flops_per_step": block_flops,
-                   "l2": "inputs larger than L2: each layer reads 128 MiB of q/k/v and writes 64 MiB",
-                   "parallelism": f"independent replicas x{world}"},
+        "config": block_config(cfg, world, block_flops),
         "roofline": roofline,
         "kernels": kernels,
         "layer_kinds": layer_kinds,
@@ -617,33 +629,41 @@ def run_gpu(args, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "decode": decode,
+        "long_blocks": long_blocks,
     }
     return line
 
 
-def run_decode(args, dev, stream, world, pk, pk_kind):
+def run_decode(args, dev, stream, rank, world, pk, pk_kind):
+    """Six g3attn_decode calls on the 64-sequence batch; under torchrun the
+    batch is split by sequence (shard.sequence_shard) and the rate counts the
+    whole batch's bytes over the slowest rank's time (strong scaling)."""
     import torch
     import global_gqa_b200 as g3
     cfg = inputs.DECODE_B64
     blk = cfg.block()
-    lens = inputs.decode_lengths(cfg.B, cfg.len_lo, cfg.len_hi, cfg.seed)
+    lens_all = inputs.decode_lengths(cfg.B, cfg.len_lo, cfg.len_hi, cfg.seed)
+    b0, b1 = shard.sequence_shard(cfg.B, world, rank)
+    B = b1 - b0
+    lens = lens_all[b0:b1]
     sl = lens.to(dev)
     caches = []
     for li, L in enumerate(blk):
         if L.kind == 0:
-            kc = torch.empty(cfg.B, cfg.Hkv, cfg.window, cfg.D, dtype=torch.bfloat16, device=dev)
+            kc = torch.empty(B, cfg.Hkv, cfg.window, cfg.D, dtype=torch.bfloat16, device=dev)
         else:
-            kc = torch.empty(cfg.B, cfg.Hkv, cfg.global_capacity, cfg.D, dtype=torch.bfloat16, device=dev)
+            kc = torch.empty(B, cfg.Hkv, cfg.global_capacity, cfg.D, dtype=torch.bfloat16, device=dev)
         vc = torch.empty_like(kc)
-        inputs.device_fill_normal_bf16(kc, inputs.seed_for(cfg.seed, li, inputs.T_KC))
-        inputs.device_fill_normal_bf16(vc, inputs.seed_for(cfg.seed, li, inputs.T_VC))
-        x = {k: v.to(dev) for k, v in inputs.decode_step_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, seed=cfg.seed,
-                                                               layer=li).items()}
+        inputs.device_fill_normal_bf16(kc, inputs.seed_for(cfg.seed, li, inputs.T_KC) + b0)
+        inputs.device_fill_normal_bf16(vc, inputs.seed_for(cfg.seed, li, inputs.T_VC) + b0)
+        step_in = inputs.decode_step_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, seed=cfg.seed, layer=li)
+        x = {k: (v[b0:b1] if v.dim() == 3 else v).contiguous().to(dev) for k, v in step_in.items()}
         x["out"] = torch.empty_like(x["q"])
         caches.append((L, kc, vc, x))
-    ws = torch.empty(g3.decode_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.len_hi), dtype=torch.uint8,
+    ws = torch.empty(g3.decode_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.D, cfg.len_hi), dtype=torch.uint8,
                      device=dev)
     step_bytes = sum(metrics.decode_kv_bytes(lens.numpy(), cfg.Hkv, cfg.D, L.kind, L.window) for L in blk)
+    all_bytes = sum(metrics.decode_kv_bytes(lens_all.numpy(), cfg.Hkv, cfg.D, L.kind, L.window) for L in blk)
 
     def step():
         for L, kc, vc, x in caches:
@@ -671,7 +691,7 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
         torch.distributed.barrier()
     trace = g3.trace_collect()
     ms = max_over_ranks(e0.elapsed_time(e1), dev)
-    gbs = weak_scaling_rate(step_bytes, args.steps, world, ms) / 1e9
+    gbs = all_bytes * args.steps / (ms * 1e-3) / 1e9
     n_split, split_ms = trace.get("decode_split", (0, 0.0))
     ach = step_bytes * n_traced(args.steps) / (split_ms * 1e-3) / 1e9 if split_ms > 0 else None
     del caches
@@ -679,7 +699,9 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
     return {
         "metric": "decode KV GB/s (5:1 block)", "value": gbs, "unit": "GB/s", "ms_per_step": ms / args.steps,
         "config": {"workload": cfg.name, "batch": cfg.B, "context": f"U[{cfg.len_lo},{cfg.len_hi}]",
-                   "kv_bytes_per_step": step_bytes, "l2": "inputs larger than L2 (~38 GB of cache read per step)"},
+                   "kv_bytes_per_step": all_bytes, "l2": "inputs larger than L2 (~38 GB of cache read per step)",
+                   "parallelism": f"batch split by sequence over {world} rank(s)", "sequences_per_rank": B},
+        "scaling": "strong",
         "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": (ach / pk["hbm_gbs"]) if ach else None,
                      "traffic": decode_traffic_per_launch(step_bytes / len(blk)), "kernel": "decode_split",
@@ -688,6 +710,171 @@ def run_decode(args, dev, stream, world, pk, pk_kind):
         "kernels": {k: {"launches": v[0], "ms": v[1]} for k, v in trace.items()},
         "gpu_launches": launches_in_timed_region(trace, args.steps),
     }
+
+
+# ------------------------------------------- mixed text+image and 128K blocks
+LONG_CONFIGS = (inputs.MIXED_32K, inputs.LONG_128K)
+
+
+def long_block_spans(cfg):
+    """Image spans of the workload: one set per sequence, the same in every
+    layer of the block (images sit at fixed token positions)."""
+    return inputs.image_spans(cfg.B, cfg.S, cfg.n_spans, cfg.seed, 0)
+
+
+def run_long_blocks(args, dev, stream, rank, world, pk, pk_kind):
+    """Times the six g3attn_prefill calls of the mixed text+image block (2 x
+    32768 tokens, 8 images of 256 tokens per sequence) and of the 128K block,
+    each outside the headline timed region; inputs are generated on the device.
+    Under torchrun the kv heads are split over the ranks (shard.kv_head_shard)
+    and the rate counts the whole block over the slowest rank (strong scaling)."""
+    import torch
+    import global_gqa_b200 as g3
+    res = {}
+    for cfg_all in LONG_CONFIGS:
+        G = cfg_all.Hq // cfg_all.Hkv
+        sh = shard.kv_head_shard(cfg_all.Hkv, G, world, rank)
+        Hkv_r = sh["kv"][1] - sh["kv"][0]
+        if Hkv_r == 0:
+            # a rank without kv heads still takes the same collective steps
+            torch.distributed.barrier()
+            max_over_ranks(0.0, dev)
+            torch.distributed.barrier()
+            continue
+        cfg = inputs.PrefillConfig(cfg_all.name, cfg_all.B, cfg_all.S, Hkv_r * G, Hkv_r, cfg_all.D, cfg_all.n_spans,
+                                   cfg_all.global_interp, cfg_all.seed + 7919 * sh["kv"][0])
+        blk = cfg.block()
+        spans = long_block_spans(cfg)
+        spans_d = None if spans is None else spans.to(dev)
+        layers = []
+        for li, L in enumerate(blk):
+            x = {}
+            for name, shape, tid in (("q", (cfg.B, cfg.S, cfg.Hq, cfg.D), inputs.T_Q),
+                                     ("k", (cfg.B, cfg.S, cfg.Hkv, cfg.D), inputs.T_K),
+                                     ("v", (cfg.B, cfg.S, cfg.Hkv, cfg.D), inputs.T_V)):
+                x[name] = inputs.device_fill_normal_bf16(torch.empty(shape, dtype=torch.bfloat16, device=dev),
+                                                         inputs.seed_for(cfg.seed, li, tid))
+            x["q_gamma"] = inputs.gamma(cfg.D, cfg.seed, li, inputs.T_QG).to(dev)
+            x["k_gamma"] = inputs.gamma(cfg.D, cfg.seed, li, inputs.T_KG).to(dev)
+            x["positions"] = inputs.positions(cfg.B, cfg.S).to(dev)
+            x["out"] = torch.empty_like(x["q"])
+            layers.append((L, x))
+        ws = torch.empty(g3.prefill_workspace_size(cfg.B, cfg.S, cfg.Hq, cfg.Hkv, cfg.D), dtype=torch.uint8,
+                         device=dev)
+        flops = metrics.block_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, blk,
+                                    None if spans is None else spans.numpy())
+        flops_all = flops * cfg_all.Hq / cfg.Hq
+
+        def call(L, x):
+            g3.prefill(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind, L.window,
+                       L.rope_base, L.interp, spans_d, out=x["out"], ws=ws, stream=stream)
+
+        for L, x in layers:  # warm-up block
+            call(L, x)
+        if g3.check_device_error(ws) != 0:
+            raise RuntimeError(f"device error in the {cfg.name} warm-up")
+        reps = 3 if cfg.S > 65536 else 5
+        g3.trace_collect()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(reps):
+            g3.trace_enable(i == 0)  # the first block carries the kernel trace
+            for L, x in layers:
+                call(L, x)
+        g3.trace_enable(False)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        tr = g3.trace_collect()
+        if g3.check_device_error(ws) != 0:
+            raise RuntimeError(f"device error in the {cfg.name} timing")
+        ms = max_over_ranks(e0.elapsed_time(e1) / reps, dev)
+        if world > 1:
+            torch.distributed.barrier()
+        n_attn, attn_ms = tr.get("prefill_attention", (0, 0.0))
+        ach = flops / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
+        # per layer kind: one local and the global layer, traced alone
+        kinds = {}
+        for li in (0, len(blk) - 1):
+            L, x = layers[li]
+            f = metrics.layer_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, L.kind, L.window,
+                                    None if spans is None else spans.numpy())
+            g3.trace_collect()
+            g3.trace_enable(True)
+            call(L, x)
+            g3.trace_enable(False)
+            t = g3.trace_collect()
+            na, ma = t.get("prefill_attention", (1, 0.0))
+            npro, mpro = t.get("prefill_prologue", (1, 0.0))
+            kinds["local" if L.kind == 0 else "global"] = {
+                "flops": f, "attention_us": 1e3 * ma / na, "attention_tflops": f / (ma / na * 1e-3) / 1e12,
+                "prologue_us": 1e3 * mpro / npro}
+        res[cfg.name] = {
+            "workload": cfg.name,
+            "config": {"batch": cfg.B, "seq_len": cfg.S, "q_heads": cfg_all.Hq, "kv_heads": cfg_all.Hkv,
+                       "head_dim": cfg.D, "image_spans_per_sequence": cfg.n_spans,
+                       "global_interp": cfg.global_interp, "unmasked_flops_per_block": flops_all,
+                       "l2": "inputs far larger than L2", "inputs": "N(0,1) bf16 generated on the device",
+                       "parallelism": f"kv heads split over {world} rank(s)", "kv_heads_per_rank": cfg.Hkv},
+            "scaling": "strong",
+            "ms_per_block": ms, "tflops": flops_all / (ms * 1e-3) / 1e12, "blocks_timed": reps,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": (ach / pk["bf16_tflops"]) if ach else None, "traffic": None,
+                         "kernel": "prefill_attention", "peak_kind": f"{pk_kind} dense bf16 burst",
+                         "launches": n_attn, "avg_launch_ms": attn_ms / max(n_attn, 1)},
+            "kernels": {k: {"launches": v[0], "ms": v[1]} for k, v in tr.items()},
+            "layer_kinds": kinds,
+            "gpu_launches": sum(v[0] for v in tr.values()) * reps,
+        }
+        del layers, ws, x
+        torch.cuda.empty_cache()
+    return res
+
+
+def oracle_long_baselines(long_res: dict, budget_s: float) -> None:
+    """The oracle timed as it stands on sampled query rows of every layer of the
+    mixed and 128K blocks, on one GQA group (2 query heads, 1 kv head) of the
+    same sequences and spans; its FLOP rate is extrapolated to the whole block
+    by the unmasked-pair count."""
+    from oracle import attention as O
+    for cfg in LONG_CONFIGS:
+        r = long_res.get(cfg.name) if long_res else None
+        if not r:
+            continue
+        blk = cfg.block()
+        spans = long_block_spans(cfg)
+        sp = None if spans is None else spans.numpy()
+        rng = np.random.default_rng(5)
+        flops, secs, nrows, li = 0.0, 0.0, 0, 0
+        per_layer = max(budget_s / len(blk), 0.5)
+        for li, L in enumerate(blk):
+            x = inputs.prefill_layer_inputs(cfg.B, cfg.S, 2, 1, cfg.D, seed=cfg.seed, layer=li)
+            lo, hi = [], []
+            for b in range(cfg.B):
+                a, c = metrics.row_intervals(cfg.S, L.kind, L.window, None if sp is None else sp[b])
+                lo.append(a)
+                hi.append(c)
+            t_layer = 0.0
+            while t_layer < per_layer:
+                rows = np.sort(rng.choice(cfg.S, 128, replace=False))
+                t0 = time.perf_counter()
+                O.prefill_rows(x["q"], x["k"], x["v"], x["q_gamma"], x["k_gamma"], x["positions"], L.kind,
+                               L.window, L.rope_base, L.interp, spans, rows=rows)
+                dt = time.perf_counter() - t0
+                t_layer += dt
+                secs += dt
+                flops += 4.0 * cfg.D * 2 * sum(float(np.sum(hi[b][rows] - lo[b][rows] + 1)) for b in range(cfg.B))
+                nrows += rows.size * cfg.B
+        rate = flops / secs
+        r["cpu_baseline"] = {
+            "value": rate / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "seconds": secs,
+            "extrapolated_s_per_block": r["config"]["unmasked_flops_per_block"] / rate,
+            "sample": f"{nrows} query rows (groups of 128, every layer) of one GQA group (2 query heads, 1 kv head) "
+                      f"of the {cfg.name} sequences, float64 numpy; the block time is extrapolated by "
+                      f"unmasked-pair count"}
 
 
 # ---------------------------------------------------------- reference arm
@@ -705,8 +892,8 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "batch": cfg.B, "seq_len": cfg.S, "q_heads": cfg.Hq,
-                       "kv_heads": cfg.Hkv, "head_dim": cfg.D},
+            "config": block_config(cfg, int(os.environ.get("WORLD_SIZE", "1")),
+                                   metrics.block_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, cfg.block())),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -748,6 +935,7 @@ def main():
                                           f"{inputs.BLOCK_8K.name} block, float64 numpy"}
         if args.extras and args.cpu_budget > 0:
             oracle_extras_baselines(line)
+            oracle_long_baselines(line.get("long_blocks"), args.cpu_budget / 2)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -143,6 +143,25 @@ def workspace(nbytes: int, device, tag: str = "default", stream=None):
     return buf
 
 
+def release_workspaces(device=None, stream=None) -> int:
+    """Drops the cached workspaces (all of them, or those of one device and/or
+    stream) so torch can reuse their memory; returns how many were dropped.
+    A server that makes a stream per request calls this when the stream is
+    retired.  Work already queued keeps its buffer alive through torch's
+    stream-ordered allocator."""
+    torch = _torch()
+    dev = None
+    if device is not None:
+        dev = torch.device(device)
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+    sid = None if stream is None else int(stream.cuda_stream)
+    drop = [k for k in _workspaces if (dev is None or k[0] == str(dev)) and (sid is None or k[2] == sid)]
+    for k in drop:
+        del _workspaces[k]
+    return len(drop)
+
+
 def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
@@ -316,7 +335,9 @@ def decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, seq_lens, max_se
     dev = q.device
     _on_device(dev, k_new=k_new, v_new=v_new, q_gamma=q_gamma, k_gamma=k_gamma, k_cache=k_cache,
                v_cache=v_cache, seq_lens=seq_lens, out=out)
-    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, max_seq_len), dev, stream=stream)
+    # Decode keeps its own cached workspace: its launch clears the error word,
+    # which would otherwise erase a prefill's unread device error.
+    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, max_seq_len), dev, tag="decode", stream=stream)
     with torch.cuda.device(dev):
         st = lib().g3attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_gamma), _ptr(k_gamma),
                                  _ptr(k_cache), _ptr(v_cache), cap, _ptr(seq_lens), int(max_seq_len),

@@ -393,6 +393,7 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   ap.G = G;
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
+  ap.chains = layer_kind == G3_LAYER_LOCAL ? 1 : 0;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill attention: %s", cudaGetErrorString(e));
@@ -532,6 +533,7 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
   ap.G = G;
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
+  ap.chains = layer_kind == G3_LAYER_LOCAL ? 1 : 0;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk attention: %s", cudaGetErrorString(e));
@@ -701,9 +703,11 @@ g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new, con
   if (G != 1 && G != 2 && G != 4) return fail(G3_ERR_UNSUPPORTED, "decode: group size %d not built (1, 2, 4)", G);
   if ((size_t)B * Hkv * cache_capacity * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "decode: cache too large");
 
+  // The split-KV partials are laid out for the slots a query can see: on a
+  // local layer at most min(max_seq_len, window), however long the sequence.
   DecodeWs w;
   const int visible_max = layer_kind == G3_LAYER_LOCAL ? std::min(max_seq_len, window) : max_seq_len;
-  decode_ws(B, Hq, Hkv, D, max_seq_len, &w);
+  decode_ws(B, Hq, Hkv, D, visible_max, &w);
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(G3_ERR_WORKSPACE, "decode: workspace NULL or not 256-byte aligned");
   if (workspace_bytes < w.total)

@@ -14,8 +14,10 @@
 //   * every GPU that loads the library holds kStaticScratchBytes (16 MiB) of
 //     device memory for this array until the process exits;
 //   * sizes whose scratch would exceed the array are rejected with
-//     G3_ERR_UNSUPPORTED (roughly B * Hq * ceil(max_seq_len / 512) * (D + 2) * 4
-//     bytes plus a small header, see g3attn_decode_workspace_size);
+//     G3_ERR_UNSUPPORTED (roughly B * Hq * ceil(n / 512) * (D + 2) * 4 bytes
+//     plus a small header, n = max_seq_len on a global layer and
+//     min(max_seq_len, window) on a local one; see
+//     g3attn_decode_workspace_size);
 //   * all calls on a device share the one array and it keeps the last call's
 //     contents: calls that may overlap on the GPU (different streams without
 //     ordering between them) race on it and must be serialised by the caller;
@@ -71,7 +73,10 @@ extern "C" g3_status g3attn_decode_no_alloc(const void* q, const void* k_new, co
                                             int32_t max_seq_len, g3_layer_kind layer_kind, int32_t window,
                                             float rope_base, float interp_factor, int32_t B, int32_t Hq,
                                             int32_t Hkv, int32_t D, void* out, void* stream) {
-  const size_t need = g3attn_decode_workspace_size(B, Hq, Hkv, D, max_seq_len);
+  // Scratch as g3attn_decode lays it out: split-KV partials for the slots a
+  // query can see (min(max_seq_len, window) on a local layer).
+  const int32_t visible = (layer_kind == G3_LAYER_LOCAL && window >= 1 && window < max_seq_len) ? window : max_seq_len;
+  const size_t need = g3attn_decode_workspace_size(B, Hq, Hkv, D, visible);
   if (need == 0) {
     // Invalid sizes: let the regular entry point report them (nothing runs).
     return g3attn_decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, cache_capacity, seq_lens,

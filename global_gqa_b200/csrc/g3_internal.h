@@ -56,6 +56,7 @@ struct AttnParams {
   int B, S, Hq, Hkv, G;
   int n_qtiles;
   int n_groups;        // G / heads_per_cta
+  int chains;          // sliding-window layer: the persistent two-chain kernel may serve it (head dim 128)
   float scale_log2;    // log2(e) / sqrt(D)
 };
 

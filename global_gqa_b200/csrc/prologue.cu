@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(ProloguePa
       }
       p.lo[bt] = lo - p.key_base;
       p.hi[bt] = hi - p.key_base;
+      // A filled cache is read back by decode, which rotates each new token by
+      // its index: keys cached here must have been rotated by theirs.
+      if (p.k_cache != nullptr && p.positions[bt] != ta) record_error(p.err, kErrInvalid, 101);
       if (t == 0 && p.n_spans > 0) {
         // Sorted, disjoint, inside the sequence, and (chunked prefill) not
         // holding tokens on both sides of the chunk's first or last boundary.

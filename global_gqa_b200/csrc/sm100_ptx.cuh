@@ -230,34 +230,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
-// Register reallocation between warpgroups (all warps of a warpgroup execute
-// the same call).
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // --------------------------------------------------------------- math bits
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x0 and 2^x1 with one exp-unit operation: both arguments are rounded to
-// f16 (error <= |x| * 2^-11, below the bf16 rounding the probabilities get
-// afterwards) and exponentiated as an f16 pair; the results come back as fp32.
-__device__ __forceinline__ void ex2_pair_f16(float x0, float x1, float& p0, float& p1) {
-  uint32_t h, e;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-  asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
-      : "=f"(p0), "=f"(p1)
-      : "r"(e));
 }
 
 // (a0, a1) * (b, b) + (c, c) as one packed fp32x2 operation.
@@ -283,30 +260,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// Coefficients of a cubic approximating 2^f on [-0.5, 0.5] with the constant
-// term held at exactly 1 (so integer x gives exactly 2^x), fitted for this
-// library by iteratively reweighted least squares on the relative error
-// (max relative error 1.02e-4 when evaluated in fp32 with fma).
-constexpr float kExp2C0 = 1.0f;
-constexpr float kExp2C1 = 0.6932829022407532f;
-constexpr float kExp2C2 = 0.24221062660217285f;
-constexpr float kExp2C3 = 0.05500869080424309f;
-
-// 2^x on the FMA/ALU pipes, for x <= 64: x is split as n + f with n = rint(x)
-// obtained by adding 1.5 * 2^23 (the integer lands in the low mantissa bits),
-// f = x - n in [-0.5, 0.5]; 2^f comes from the cubic and n is added to its
-// exponent field.  Inputs below -125 (masked scores are -inf) give exactly 0.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float xc = fmaxf(x, -126.f);
-  const float shift = 12582912.f;  // 1.5 * 2^23
-  const float t = xc + shift;
-  const float n = t - shift;
-  const float f = xc - n;
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -125.f ? 0.f : r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

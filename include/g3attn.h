@@ -89,7 +89,11 @@ size_t g3attn_prefill_workspace_size(int32_t B, int32_t S, int32_t Hq, int32_t H
  *              later g3attn_decode.  GLOBAL: token t goes to slot t and
  *              cache_capacity >= S.  LOCAL: a ring of cache_capacity == window
  *              slots; token t goes to slot t % window and only the last
- *              min(S, window) tokens are written.  Both NULL to skip.
+ *              min(S, window) tokens are written.  Both NULL to skip.  A
+ *              filled cache is read by g3attn_decode, which rotates each new
+ *              token by its index, so with a cache positions[b, t] must be t;
+ *              any other position is recorded as G3_ERR_INVALID_ARG for
+ *              g3attn_check_device_error() (the cache is still written).
  *   workspace  >= g3attn_prefill_workspace_size(B, S, Hq, Hkv, D) bytes
  */
 g3_status g3attn_prefill(const void* q, const void* k, const void* v,
@@ -120,7 +124,10 @@ size_t g3attn_prefill_chunk_workspace_size(int32_t B, int32_t C, int32_t Hq, int
  *   q, k, v    bf16 [B, C, Hq|Hkv, D]  raw projections of the chunk's tokens
  *   q_gamma, k_gamma, layer_kind, window, rope_base, interp_factor
  *              as for g3attn_prefill
- *   positions  int32 [B, C]  RoPE positions of the chunk's tokens
+ *   positions  int32 [B, C]  RoPE positions of the chunk's tokens: start + t
+ *              for token t (the cached keys are rotated by their index, as
+ *              decode expects); any other value is recorded as
+ *              G3_ERR_INVALID_ARG for g3attn_check_device_error()
  *   k_cache, v_cache bf16 [B, Hkv, cache_capacity, D], required: rotated keys
  *              and values of tokens 0 .. start-1 as g3attn_prefill (with
  *              caches) or earlier chunks left them.  GLOBAL: token t in slot t,
@@ -215,7 +222,9 @@ g3_status g3attn_soft_tokens(const void* patches, const float* gamma, int32_t B,
                              int32_t grid_w, int32_t F, int32_t pool, void* out, void* stream);
 
 /* ------------------------------------------------------------------- decode
- * Bytes of workspace g3attn_decode needs (0 if the sizes are invalid).
+ * Bytes of workspace g3attn_decode needs (0 if the sizes are invalid).  The
+ * figure for max_seq_len covers both layer kinds; a LOCAL layer needs only the
+ * figure for min(max_seq_len, window), the most slots a query there can see.
  */
 size_t g3attn_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
                                     int32_t max_seq_len);
@@ -236,7 +245,8 @@ size_t g3attn_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t 
  *              and L <= cache_capacity for GLOBAL layers
  *   max_seq_len host-side upper bound of seq_lens, used to size the launch
  *   out        bf16 [B, Hq, D]
- *   workspace  >= g3attn_decode_workspace_size(B, Hq, Hkv, D, max_seq_len)
+ *   workspace  >= g3attn_decode_workspace_size(B, Hq, Hkv, D, n) bytes, n =
+ *              max_seq_len (GLOBAL) or min(max_seq_len, window) (LOCAL)
  * A sequence whose length is out of range gets a zero output row, its cache is
  * left untouched, and G3_ERR_INVALID_ARG is recorded for
  * g3attn_check_device_error().
@@ -261,8 +271,8 @@ g3_status g3attn_decode(const void* q, const void* k_new, const void* v_new,
  * Same arguments and results as g3attn_decode, minus the workspace: the
  * scratch lives in a 16 MiB device array inside the library, which every GPU
  * that loads the library keeps until the process exits.  The call allocates
- * nothing.  Sizes whose scratch (g3attn_decode_workspace_size) exceeds
- * 16 MiB return G3_ERR_UNSUPPORTED with a message in g3attn_last_error().
+ * nothing.  Sizes whose scratch (the workspace g3attn_decode would need)
+ * exceeds 16 MiB return G3_ERR_UNSUPPORTED with a message in g3attn_last_error().
  * All calls on a device share the array and it keeps the last call's
  * contents, so calls that may overlap on the GPU race and must be ordered by
  * the caller.  The first call on each device looks up the array's address;

@@ -41,3 +41,17 @@ def test_trace_sampling_counts():
     trace = {"prefill_prologue": (6 * bench.n_traced(steps), 1.0),
              "prefill_attention": (6 * bench.n_traced(steps), 9.0)}
     assert bench.launches_in_timed_region(trace, steps) == 12 * steps
+
+
+def test_long_block_spans_are_the_workloads():
+    # the mixed block: 8 images of 256 tokens per sequence, sorted, disjoint and
+    # inside the sequence; the same set serves every layer of the block
+    import numpy as np
+    import inputs
+    cfg = inputs.MIXED_32K
+    sp = bench.long_block_spans(cfg).numpy()
+    assert sp.shape == (cfg.B, cfg.n_spans, 2)
+    assert ((sp[:, :, 1] - sp[:, :, 0]) == 256).all()
+    assert (sp[:, 1:, 0] >= sp[:, :-1, 1]).all() and sp.min() >= 0 and sp.max() <= cfg.S
+    assert np.array_equal(sp, bench.long_block_spans(cfg).numpy())
+    assert bench.long_block_spans(inputs.LONG_128K) is None

@@ -23,6 +23,12 @@ def test_reference_arm_line():
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 0
     assert d["config"]["workload"] == "gemma3_27b_block_s8192"
+    # the GPU arm prints the same config object for the same workload
+    import bench
+    import inputs
+    from global_gqa_b200 import metrics
+    cfg = inputs.BLOCK_8K
+    assert d["config"] == bench.block_config(cfg, 1, metrics.block_flops(cfg.B, cfg.S, cfg.Hq, cfg.D, cfg.block()))
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -77,3 +77,15 @@ def test_workspace_cache_is_per_device_and_stream(monkeypatch):
     c = g3.workspace(4096, "cuda:0")
     assert c is not a and c.numel() >= 4096                      # grown on demand
     assert g3.workspace(100, "cuda:0") is c
+
+
+def test_release_workspaces_drops_one_stream_or_all(monkeypatch):
+    monkeypatch.setattr(g3, "_torch", lambda: _FakeTorch)
+    monkeypatch.setattr(g3, "_workspaces", {})
+    a = g3.workspace(512, "cuda:0")
+    b = g3.workspace(512, "cuda:0", stream=_FakeStream(7))
+    g3.workspace(512, "cuda:0", tag="decode", stream=_FakeStream(7))
+    assert g3.release_workspaces(stream=_FakeStream(7)) == 2     # both tags of that stream
+    assert g3.workspace(512, "cuda:0") is a                       # the other stream's buffer stays
+    assert g3.workspace(512, "cuda:0", stream=_FakeStream(7)) is not b
+    assert g3.release_workspaces() == 2 and g3._workspaces == {}

@@ -49,7 +49,7 @@ def _run_case(B, Hq, Hkv, D, lens, kind, W, base, interp, seed=0, layer=0, cap=N
     sl = torch.tensor(lens, dtype=torch.int32, device=dev())
     out = g3.decode(xd["q"], xd["k_new"], xd["v_new"], xd["q_gamma"], xd["k_gamma"], kcd, vcd, sl, max_len,
                     kind, W, base, interp)
-    assert g3.check_device_error(g3.workspace(0, dev())) == 0
+    assert g3.check_device_error(g3.workspace(0, dev(), tag="decode")) == 0
     ref, k_hat = O.decode(x["q"], x["k_new"], x["v_new"], x["q_gamma"], x["k_gamma"], lens, hk, hv, starts,
                           kind, W, base, interp)
     assert_close(out, ref)
@@ -177,7 +177,7 @@ def test_decode_full_size_sampled():
         xd = to_dev(x)
         out = g3.decode(xd["q"], xd["k_new"], xd["v_new"], xd["q_gamma"], xd["k_gamma"], kc, vc, sl,
                         cfg.len_hi, L.kind, L.window, L.rope_base, L.interp)
-        assert g3.check_device_error(g3.workspace(0, dev())) == 0
+        assert g3.check_device_error(g3.workspace(0, dev(), tag="decode")) == 0
         sub = {k: v[check] for k, v in x.items() if k in ("q", "k_new", "v_new")}
         ref, _ = O.decode(sub["q"], sub["k_new"], sub["v_new"], x["q_gamma"], x["k_gamma"], lens[check].numpy(),
                           hk, hv, starts, L.kind, L.window, L.rope_base, L.interp)
@@ -201,7 +201,7 @@ def test_decode_medium_global():
     xd = to_dev(x)
     out = g3.decode(xd["q"], xd["k_new"], xd["v_new"], xd["q_gamma"], xd["k_gamma"], kc, vc, sl, cap, O.GLOBAL,
                     cap, 1e6, 8.0)
-    assert g3.check_device_error(g3.workspace(0, dev())) == 0
+    assert g3.check_device_error(g3.workspace(0, dev(), tag="decode")) == 0
     check = [0, 3, 7]
     hk = [kc[b][:, :int(lens[b]) - 1].permute(1, 0, 2).cpu() for b in check]
     hv = [vc[b][:, :int(lens[b]) - 1].permute(1, 0, 2).cpu() for b in check]

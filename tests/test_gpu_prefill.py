@@ -148,6 +148,22 @@ def test_bad_spans_reported_on_device():
     assert g3.check_device_error(ws) == 0   # read-and-clear
 
 
+def test_cache_fill_with_positions_other_than_token_index_is_reported():
+    """Decode rotates a new token by its index, so a prefill that fills a cache
+    must have positions[b, t] == t; the prologue records anything else."""
+    B, S, Hq, Hkv, D, W = 1, 300, 2, 1, 64, 128
+    xc = inputs.prefill_layer_inputs(B, S, Hq, Hkv, D, seed=2)
+    xc["positions"] = (xc["positions"] + 5).contiguous()
+    xd = to_dev(xc)
+    ws = torch.empty(g3.prefill_workspace_size(B, S, Hq, Hkv, D), dtype=torch.uint8, device=dev())
+    kc = torch.zeros(B, Hkv, W, D, dtype=torch.bfloat16, device=dev())
+    vc = torch.zeros_like(kc)
+    run_prefill(xd, LOC, W, 1e4, 1.0, return_lse=False, ws=ws, k_cache=kc, v_cache=vc)
+    assert g3.check_device_error(ws) == 1
+    run_prefill(xd, LOC, W, 1e4, 1.0, return_lse=False, ws=ws)   # no cache: any positions are fine
+    assert g3.check_device_error(ws) == 0
+
+
 @pytest.mark.parametrize("kind", [LOC, GLB], ids=["local", "global"])
 def test_prefill_1b_shapes_32k(kind):
     """Gemma 3 1B attention shapes (4 query heads, 1 kv head, head_dim 256) at a

@@ -71,6 +71,32 @@ def test_decode_no_alloc_matches_workspace_decode(kind, W, base, interp, lens, c
         assert torch.equal(kc, kc_ref) and torch.equal(vc, vc_ref)
 
 
+def test_decode_no_alloc_local_layer_at_batched_decode_sizes():
+    """A local layer of the 64-sequence decode (32/16 heads, contexts up to 128K):
+    a query sees at most the 1024 ring slots, so the scratch is a couple of MB
+    whatever max_seq_len is, and the call is accepted."""
+    dev = torch.device("cuda", 0)
+    B, Hq, Hkv, D, W, max_len = 64, 32, 16, 128, 1024, 131072
+    x = {k: v.to(dev) for k, v in inputs.decode_step_inputs(B, Hq, Hkv, D, seed=4, layer=0).items()}
+    kc0 = torch.empty(B, Hkv, W, D, dtype=torch.bfloat16, device=dev)
+    vc0 = torch.empty_like(kc0)
+    inputs.device_fill_normal_bf16(kc0, 7)
+    inputs.device_fill_normal_bf16(vc0, 8)
+    sl = inputs.decode_lengths(B, 4096, max_len, seed=4).to(dev)
+    kc_ref, vc_ref = kc0.clone(), vc0.clone()
+    ref = g3.decode(x["q"], x["k_new"], x["v_new"], x["q_gamma"], x["k_gamma"], kc_ref, vc_ref, sl, max_len,
+                    0, W, 1e4, 1.0)
+    torch.cuda.synchronize()
+    kc, vc = kc0.clone(), vc0.clone()
+    for call in range(2):
+        out = torch.full((B, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+        st = _call_no_alloc(x, kc, vc, sl, max_len, 0, W, 1e4, 1.0, out)
+        assert st == 0, g3.lib().g3attn_last_error()
+        torch.cuda.synchronize()
+        _close(out, ref)
+        assert torch.equal(kc, kc_ref) and torch.equal(vc, vc_ref)
+
+
 def test_decode_no_alloc_rejects_sizes_beyond_its_array():
     dev = torch.device("cuda", 0)
     B, Hq, Hkv, D = 64, 32, 16, 128
