@@ -245,6 +245,19 @@ bool bwd_ws(int B, int S, int Hq, int Hkv, int D, BwdWs* w) {
 
 void g3::set_last_error(const char* msg) { g_last_error = msg; }
 
+#ifdef G3_FAULT_INJECT
+// Test-only build (never the product library): the next prefill launch makes
+// the MMA thread of CTA `cta` skip its first "S ready" arrival, so that the
+// softmax warps' bounded wait runs out and the kernel reports G3_ERR_TIMEOUT.
+namespace {
+std::atomic<int> g_withhold_cta{-1};
+}
+extern "C" void g3attn_test_withhold_s_commit(int32_t cta) { g_withhold_cta.store(cta); }
+static int take_withhold_cta() { return g_withhold_cta.exchange(-1); }
+#else
+static int take_withhold_cta() { return -1; }
+#endif
+
 extern "C" {
 
 const char* g3attn_status_string(g3_status s) {
@@ -394,6 +407,7 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
   ap.chains = layer_kind == G3_LAYER_LOCAL ? 1 : 0;
+  ap.withhold_cta = take_withhold_cta();
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill attention: %s", cudaGetErrorString(e));
@@ -534,6 +548,7 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
   ap.chains = layer_kind == G3_LAYER_LOCAL ? 1 : 0;
+  ap.withhold_cta = take_withhold_cta();
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk attention: %s", cudaGetErrorString(e));

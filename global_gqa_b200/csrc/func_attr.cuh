@@ -5,6 +5,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <utility>
 
 namespace g3 {
 
@@ -23,6 +24,26 @@ cudaError_t ensure_dynamic_smem(Kernel* kernel, int bytes, std::atomic<uint64_t>
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_acq_rel);
   return e;
+}
+
+// Launches `kernel` as a programmatic dependent of the previous work in
+// `stream`: its CTAs may start while that kernel drains, and must call
+// griddep_wait() before reading anything it wrote.
+template <class... Params, class... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace g3

@@ -57,6 +57,7 @@ struct AttnParams {
   int n_qtiles;
   int n_groups;        // G / heads_per_cta
   int chains;          // sliding-window layer: the persistent two-chain kernel may serve it (head dim 128)
+  int withhold_cta;    // test-only build: this CTA's MMA thread skips its first "S ready" arrival (-1: none)
   float scale_log2;    // log2(e) / sqrt(D)
 };
 

@@ -97,15 +97,6 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
   const int r0 = qt * 128;
   const int r_last = min(r0 + 127, p.S - 1);
 
-  const size_t rowbase = (size_t)b * p.S;
-  const int lo_first = p.lo[rowbase + r0];
-  const int hi_last = p.hi[rowbase + r_last];
-  const int lo_last = p.lo[rowbase + r_last];  // largest lo of the tile's rows
-  const int hi_first = p.hi[rowbase + r0];     // smallest hi of the tile's rows
-  const int t_begin = lo_first / 128;
-  const int n_tiles = max(hi_last / 128, t_begin) - t_begin + 1;
-  const int n_pre = min(n_tiles, NS);  // K/V tiles loaded before the CTA-wide barrier
-
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < NS; ++s) {
@@ -123,12 +114,29 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
-    // Thread 0 is also the TMA producer: start the Q tiles and the first K/V
-    // stages now, so their latency overlaps the TMEM allocation and the
-    // CTA-wide barrier below (the ring's empty barriers start released).
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
+  }
+  if (warp == 1) tmem_alloc(&bars->tmem_base, L::kTmemCols);
+
+  // Everything above is independent of the prologue's results; launched as a
+  // programmatic dependent of the prologue, the CTA waits only here for its
+  // intervals and its rotated q and k.
+  griddep_wait();
+  const size_t rowbase = (size_t)b * p.S;
+  const int lo_first = p.lo[rowbase + r0];
+  const int hi_last = p.hi[rowbase + r_last];
+  const int lo_last = p.lo[rowbase + r_last];  // largest lo of the tile's rows
+  const int hi_first = p.hi[rowbase + r0];     // smallest hi of the tile's rows
+  const int t_begin = lo_first / 128;
+  const int n_tiles = max(hi_last / 128, t_begin) - t_begin + 1;
+  const int n_pre = min(n_tiles, NS);  // K/V tiles loaded before the CTA-wide barrier
+
+  if (tid == 0) {
+    // Thread 0 is also the TMA producer: start the Q tiles and the first K/V
+    // stages now, so their latency overlaps the CTA-wide barrier below (the
+    // ring's empty barriers start released).
     mbar_arrive_expect_tx(&bars->q_full, HPC * L::kTile);
     for (int h = 0; h < HPC; ++h)
       for (int kb = 0; kb < KB; ++kb)
@@ -144,7 +152,6 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
         tma_load_4d(smem + L::kV + t * L::kTile + kb * kSwizzleBlock, &tm_v, &bars->v_full[t], kb * 64, c1, c2, b);
     }
   }
-  if (warp == 1) tmem_alloc(&bars->tmem_base, L::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -226,7 +233,10 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
             issue_pv(h, sp, t - 1 > 0);
           }
           issue_s(h, s);
-          mma_commit(&bars->s_full[h]);
+#ifdef G3_FAULT_INJECT
+          if (!(t == 0 && h == 0 && (int)blockIdx.x == p.withhold_cta))
+#endif
+            mma_commit(&bars->s_full[h]);
         }
         if (!ok) break;
         mma_commit(&bars->k_empty[s]);
@@ -438,8 +448,8 @@ static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, con
   const cudaError_t e = ensure_dynamic_smem(prefill_attention_kernel<D, HPC>, L::kAlloc, configured);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hkv * p.n_groups;
-  prefill_attention_kernel<D, HPC><<<grid, AttnRoles<HPC>::kThreads, L::kAlloc, st>>>(tq, tk, tv, to, p);
-  return cudaGetLastError();
+  return launch_dependent(prefill_attention_kernel<D, HPC>, dim3(grid), dim3(AttnRoles<HPC>::kThreads), L::kAlloc,
+                          st, tq, tk, tv, to, p);
 }
 
 cudaError_t launch_prefill_attention(const AttnParams& p, int D, int hpc, const CUtensorMap& tq,

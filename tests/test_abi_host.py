@@ -204,3 +204,15 @@ def test_block_flops_of_8k_block():
     local = 8192 * 1024 - 1023 * 1024 // 2
     glob = 8192 * 8193 // 2
     assert f == 4 * 128 * 32 * (5 * local + glob)
+
+
+def test_fault_injection_only_in_the_test_build(lib):
+    """The withheld-arrival hook and the 20 ms wait limit exist only in the
+    test-only library under _build/; the product library has neither."""
+    from global_gqa_b200 import build as B
+    assert not hasattr(lib, "g3attn_test_withhold_s_commit")
+    assert not any("FAULT" in f or "TIMEOUT" in f for f in B.FLAGS)
+    assert os.path.dirname(B.FAULT_LIB) != os.path.dirname(B.LIB)
+    path = B.build_fault_inject()
+    test_lib = ctypes.CDLL(path)
+    assert hasattr(test_lib, "g3attn_test_withhold_s_commit")
