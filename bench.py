@@ -898,6 +898,37 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_probe_layer(kind_name: str, S: int) -> dict:
+    """One 27B-shaped attention layer (B 1, 32 query / 16 kv heads, D 128) of S
+    tokens, run twice (the second call is the one a profiler captures with
+    `-s` skipping the first launches); prints its traced attention time."""
+    import torch
+    import global_gqa_b200 as g3
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kind = 0 if kind_name == "local" else 1
+    base, interp = (1e4, 1.0) if kind == 0 else (1e6, 8.0)
+    x = {}
+    for name, H, tid in (("q", 32, inputs.T_Q), ("k", 16, inputs.T_K), ("v", 16, inputs.T_V)):
+        x[name] = inputs.device_fill_normal_bf16(torch.empty(1, S, H, 128, dtype=torch.bfloat16, device=dev),
+                                                 inputs.seed_for(0, kind, tid))
+    qg, kg = inputs.gamma(128, 0, kind, inputs.T_QG).to(dev), inputs.gamma(128, 0, kind, inputs.T_KG).to(dev)
+    pos = inputs.positions(1, S).to(dev)
+    out = torch.empty_like(x["q"])
+    ws = torch.empty(g3.prefill_workspace_size(1, S, 32, 16, 128), dtype=torch.uint8, device=dev)
+    for i in range(2):
+        g3.trace_enable(i == 1)
+        g3.prefill(x["q"], x["k"], x["v"], qg, kg, pos, kind, 1024, base, interp, out=out, ws=ws)
+    torch.cuda.synchronize(dev)
+    g3.trace_enable(False)
+    if g3.check_device_error(ws) != 0:
+        raise RuntimeError("device error in the probe layer")
+    n, ms = g3.trace_collect()["prefill_attention"]
+    f = metrics.layer_flops(1, S, 32, 128, kind, 1024)
+    return {"probe_layer": kind_name, "seq_len": S, "attention_us": 1e3 * ms / n,
+            "attention_tflops": f / (ms / n * 1e-3) / 1e12}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -908,7 +939,13 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false",
                     help="skip the chunked-prefill and 1B-shape measurements")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--probe-layer", choices=["local", "global"],
+                    help="only run one 27B-shaped layer of --probe-seq tokens twice (for profiler captures)")
+    ap.add_argument("--probe-seq", type=int, default=32768)
     args = ap.parse_args()
+    if args.probe_layer:
+        print(json.dumps(run_probe_layer(args.probe_layer, args.probe_seq)), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
