@@ -388,7 +388,8 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
       !make_bshd_map(&to, out, B, S, Hq, D))
     return fail(G3_ERR_CUDA, "prefill: cuTensorMapEncodeTiled unavailable or failed");
 
-  cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
+  // Not traced: events around it would hold the prologue behind it.
+  cudaError_t e = g3::launch_error_reset(err, st);
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill: %s", cudaGetErrorString(e));
   e = traced("prefill_prologue", st, [&] { return g3::launch_prefill_prologue(pp, D, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill prologue: %s", cudaGetErrorString(e));
@@ -524,7 +525,8 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
       !make_bshd_map(&to, out, B, C, Hq, D))
     return fail(G3_ERR_CUDA, "prefill_chunk: cuTensorMapEncodeTiled unavailable or failed");
 
-  cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
+  // Not traced: events around it would hold the prologue behind it.
+  cudaError_t e = g3::launch_error_reset(err, st);
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill_chunk: %s", cudaGetErrorString(e));
   if (local && hist > 0) {
     e = traced("prefill_ring_gather", st, [&] { return g3::launch_ring_gather(rp, D, st); });
@@ -678,7 +680,8 @@ g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v, c
       !make_bshd_map(&tk, pp.k_hat, B, S, Hkv, D) || !make_bshd_map(&tv, v, B, S, Hkv, D))
     return fail(G3_ERR_CUDA, "prefill backward: cuTensorMapEncodeTiled unavailable or failed");
 
-  cudaError_t e = cudaMemsetAsync(err, 0, 8, st);
+  // Not traced: events around it would hold the prologue behind it.
+  cudaError_t e = g3::launch_error_reset(err, st);
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill backward: %s", cudaGetErrorString(e));
   e = traced("prefill_prologue", st, [&] { return g3::launch_prefill_prologue(pp, D, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill backward prologue: %s", cudaGetErrorString(e));

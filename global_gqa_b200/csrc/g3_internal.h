@@ -90,6 +90,9 @@ struct DecodeParams {
 // Launchers return the launch status; `name` receives a static kernel name
 // for tracing.
 cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st);
+// Clears a call's device-error word (err[0], err[1]) once the previous work in
+// the stream has finished, as a kernel its dependents may launch behind.
+cudaError_t launch_error_reset(int* err, cudaStream_t st);
 // Chunked prefill on a local layer: copy the ring's history rows (tokens
 // key_base .. key_base+hist-1, slot t % W) to rows 0..hist-1 of the [B, Hkv,
 // rows, D] buffers ctx_k / ctx_v, or (write_back) the chunk's last min(C, W)

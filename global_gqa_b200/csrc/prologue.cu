@@ -33,6 +33,7 @@
 #include <cstdint>
 
 #include "g3_internal.h"
+#include "func_attr.cuh"
 #include "sm100_ptx.cuh"
 
 namespace g3 {
@@ -67,6 +68,9 @@ __global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(ProloguePa
   constexpr int FPL = (H2 + 31) / 32;  // rotation angles formed per lane (FPL divides 8)
   __shared__ __align__(16) float gam[2 * D];  // q gain, then k gain
   __shared__ double inv_freq_s[H2];
+  // Launched as a programmatic dependent: nothing of the previous kernel's
+  // (it may be producing q, k, v or the positions) is read before this.
+  griddep_wait();
   for (int i = threadIdx.x; i < 2 * D; i += kRowThreads) gam[i] = i < D ? p.q_gamma[i] : p.k_gamma[i - D];
   for (int i = threadIdx.x; i < H2; i += kRowThreads) inv_freq_s[i] = p.inv_freq[i];
   __syncthreads();
@@ -214,16 +218,32 @@ __global__ void __launch_bounds__(kRowThreads, 4) qk_norm_rope_kernel(ProloguePa
   }
 }
 
+// The call's device-error reset: lets its dependent (the prologue) launch at
+// once, waits for the previous work in the stream (which may still record an
+// error in this workspace), then clears the error word and its site.
+__global__ void error_reset_kernel(int* err) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  griddep_wait();
+  if (threadIdx.x == 0) {
+    err[0] = 0;
+    err[1] = 0;
+  }
+}
+
+cudaError_t launch_error_reset(int* err, cudaStream_t st) {
+  return launch_dependent(error_reset_kernel, dim3(1), dim3(32), 0, st, err);
+}
+
 cudaError_t launch_prefill_prologue(const PrologueParams& p, int D, cudaStream_t st) {
   const long long tokens = (long long)p.B * p.S;
   long long blocks = (tokens + (kRowThreads / 32) - 1) / (kRowThreads / 32);
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (D == 128) {
-    qk_norm_rope_kernel<128><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
+    return launch_dependent(qk_norm_rope_kernel<128>, dim3((unsigned)blocks), dim3(kRowThreads), 0, st, p);
   } else if (D == 64) {
-    qk_norm_rope_kernel<64><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
+    return launch_dependent(qk_norm_rope_kernel<64>, dim3((unsigned)blocks), dim3(kRowThreads), 0, st, p);
   } else if (D == 256) {
-    qk_norm_rope_kernel<256><<<(unsigned)blocks, kRowThreads, 0, st>>>(p);
+    return launch_dependent(qk_norm_rope_kernel<256>, dim3((unsigned)blocks), dim3(kRowThreads), 0, st, p);
   } else {
     return cudaErrorInvalidValue;
   }

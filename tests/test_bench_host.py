@@ -41,6 +41,8 @@ def test_trace_sampling_counts():
     trace = {"prefill_prologue": (6 * bench.n_traced(steps), 1.0),
              "prefill_attention": (6 * bench.n_traced(steps), 9.0)}
     assert bench.launches_in_timed_region(trace, steps) == 12 * steps
+    # plus the untraced device-error reset kernel of each of the six prefill calls
+    assert bench.launches_in_timed_region(trace, steps, untraced_per_step=6) == 18 * steps
 
 
 def test_long_block_spans_are_the_workloads():
