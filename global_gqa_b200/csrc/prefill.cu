@@ -359,7 +359,8 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
         if (rescale) {
           // O is idle here: the previous P·V has completed (it was issued
           // before this tile's S) and the next one waits for p_full.
-#pragma unroll
+          // (Rolled at head dim 256, where unrolling spills.)
+#pragma unroll(D > 128 ? 1 : D / 64)
           for (int q = 0; q < D / 64; ++q) {
             float o[32];
             tmem_ld_16x256b_x8(t_lane + o_col + q * 64, o);
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
         // are clipped by the store.
         uint8_t* stage = smem + L::kQ + h * L::kTile;
         const int sw = ra & 7;  // rb = ra + 8 has the same swizzle phase
-#pragma unroll
+#pragma unroll(D > 128 ? 1 : D / 64)
         for (int q = 0; q < D / 64; ++q) {
           float o[32];
           tmem_ld_16x256b_x8(t_lane + o_col + q * 64, o);
