@@ -336,8 +336,10 @@ def decode(q, k_new, v_new, q_gamma, k_gamma, k_cache, v_cache, seq_lens, max_se
     _on_device(dev, k_new=k_new, v_new=v_new, q_gamma=q_gamma, k_gamma=k_gamma, k_cache=k_cache,
                v_cache=v_cache, seq_lens=seq_lens, out=out)
     # Decode keeps its own cached workspace: its launch clears the error word,
-    # which would otherwise erase a prefill's unread device error.
-    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, max_seq_len), dev, tag="decode", stream=stream)
+    # which would otherwise erase a prefill's unread device error.  A local
+    # layer's query sees at most `window` ring slots, which bounds its scratch.
+    visible = min(int(max_seq_len), int(window)) if layer_kind == LOCAL and window >= 1 else int(max_seq_len)
+    wsb, ws_bytes = _ws(ws, decode_workspace_size(B, Hq, Hkv, D, visible), dev, tag="decode", stream=stream)
     with torch.cuda.device(dev):
         st = lib().g3attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_gamma), _ptr(k_gamma),
                                  _ptr(k_cache), _ptr(v_cache), cap, _ptr(seq_lens), int(max_seq_len),
