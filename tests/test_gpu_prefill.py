@@ -136,6 +136,38 @@ def test_prefill_fills_cache(kind, S, W):
         assert (kcc[:, :, slot] == 7.0).all() and (vcc[:, :, slot] == 7.0).all()
 
 
+# -------------------------------------------- inputs written just before
+@pytest.mark.parametrize("kind", [LOC, GLB], ids=["local", "global"])
+def test_prefill_reads_inputs_written_just_before(kind):
+    """The prologue and attention kernels start as programmatic dependents of
+    the work before them; whatever kernel produced q, k and v right before the
+    call (here an elementwise torch kernel on the same stream, no
+    synchronisation) must be complete before they are read.  Two input sets
+    alternate over 20 calls and every output must equal its set's reference
+    bit for bit."""
+    B, S, Hq, Hkv, D = 1, 2048, 8, 4, 128
+    base, interp = (1e4, 1.0) if kind == LOC else (1e6, 8.0)
+    srcs = [to_dev(inputs.prefill_layer_inputs(B, S, Hq, Hkv, D, seed=s, layer=3)) for s in (11, 12)]
+    x = {k: (torch.empty_like(v) if k in ("q", "k", "v") else v) for k, v in srcs[0].items()}
+    refs = []
+    for src in srcs:
+        for k in ("q", "k", "v"):
+            x[k].copy_(src[k])
+        refs.append(run_prefill(x, kind, 1024, base, interp, return_lse=False).clone())
+    torch.cuda.synchronize()
+    assert not torch.equal(refs[0], refs[1])
+    outs = []
+    for i in range(20):
+        src = srcs[i % 2]
+        for k in ("q", "k", "v"):
+            torch.add(src[k], 0, out=x[k])  # a kernel on the call's stream, not a copy-engine transfer
+        outs.append(run_prefill(x, kind, 1024, base, interp, return_lse=False))
+    torch.cuda.synchronize()
+    assert g3.check_device_error(g3.workspace(0, dev())) == 0
+    for i, out in enumerate(outs):
+        assert torch.equal(out, refs[i % 2]), f"call {i} read inputs of the wrong set"
+
+
 # ------------------------------------------------------- device-side errors
 def test_bad_spans_reported_on_device():
     B, S, Hq, Hkv, D = 1, 256, 2, 1, 64
