@@ -407,7 +407,7 @@ g3_status g3attn_prefill(const void* q, const void* k, const void* v, const floa
   ap.G = G;
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
-  ap.chains = layer_kind == G3_LAYER_LOCAL ? 1 : 0;
+  ap.heavy_by_head = layer_kind == G3_LAYER_GLOBAL ? 1 : 0;
   ap.withhold_cta = take_withhold_cta();
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });
@@ -549,7 +549,7 @@ g3_status g3attn_prefill_chunk(const void* q, const void* k, const void* v, cons
   ap.G = G;
   ap.n_qtiles = (int)n_qtiles;
   ap.n_groups = G / hpc;
-  ap.chains = layer_kind == G3_LAYER_LOCAL ? 1 : 0;
+  ap.heavy_by_head = 0;  // a chunk's query tiles carry near-equal work
   ap.withhold_cta = take_withhold_cta();
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   e = traced("prefill_attention", st, [&] { return g3::launch_prefill_attention(ap, D, hpc, tq, tk, tv, to, st); });

@@ -56,7 +56,8 @@ struct AttnParams {
   int B, S, Hq, Hkv, G;
   int n_qtiles;
   int n_groups;        // G / heads_per_cta
-  int chains;          // sliding-window layer: the persistent two-chain kernel may serve it (head dim 128)
+  int heavy_by_head;   // causal layer: run the heavy query tiles kv head by kv head (see the kernel's work order)
+  int light_qtiles;    // set by the launcher: query tiles per unit left in the all-units order at the end
   int withhold_cta;    // test-only build: this CTA's MMA thread skips its first "S ready" arrival (-1: none)
   float scale_log2;    // log2(e) / sqrt(D)
 };

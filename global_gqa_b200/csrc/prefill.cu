@@ -85,10 +85,26 @@ __global__ void __launch_bounds__(AttnRoles<HPC>::kThreads, AttnRoles<HPC>::kMin
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- work item: heaviest (last) query tiles first
-  const int per_tile = p.B * p.Hkv * p.n_groups;
-  const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_tile);
-  int rem = (int)(blockIdx.x % per_tile);
+  // ---- work item.  A unit is (sequence, kv head, head group).  The grid
+  // first runs the heavy query tiles (index >= light_qtiles) unit by unit,
+  // heaviest first within each unit: the CTAs resident at one time then share
+  // one kv head's K/V in L2, which on long causal layers otherwise comes from
+  // DRAM many times over.  It ends with the light tiles of all units,
+  // heaviest first, interleaved over the units, so that the last heavy tile
+  // starts while enough light work remains to cover it.  light_qtiles =
+  // n_qtiles gives the plain heaviest-first order over all units.
+  const int units = p.B * p.Hkv * p.n_groups;
+  const int n_heavy = p.n_qtiles - p.light_qtiles;
+  const int idx = (int)blockIdx.x;
+  int qt, rem;
+  if (idx < units * n_heavy) {
+    rem = idx / n_heavy;
+    qt = p.n_qtiles - 1 - idx % n_heavy;
+  } else {
+    const int j = idx - units * n_heavy;
+    qt = p.light_qtiles - 1 - j / units;
+    rem = j % units;
+  }
   const int gp = rem % p.n_groups;
   rem /= p.n_groups;
   const int kvh = rem % p.Hkv;
@@ -440,17 +456,56 @@ size_t prefill_attention_smem_bytes(int D, int hpc) {
   return hpc == 2 ? AttnLayout<64, 2>::kAlloc : AttnLayout<64, 1>::kAlloc;
 }
 
+// Light query tiles per unit for the heavy-by-unit order of a causal layer,
+// whose query tile t visits t + 1 key tiles.  The heaviest tile of the last
+// unit starts with the light tiles of all units still to run; they hold
+// units * T^2 / 2 tile visits, and covering its n_qtiles visits on each of the
+// `resident` CTA slots needs T = sqrt(2 * n_qtiles * resident / units).
+static int light_qtiles_for(int n_qtiles, long long units, int resident) {
+  if (units <= 0 || resident <= 0) return n_qtiles;
+  const double t = std::ceil(std::sqrt(2.0 * n_qtiles * (double)resident / (double)units));
+  return t >= n_qtiles ? n_qtiles : (int)t;
+}
+
+// CTAs of `kernel` resident on the current device at once (SMs x CTAs per
+// SM), cached per device; 0 when the runtime cannot say.
+template <class Kernel>
+static int resident_ctas(Kernel* kernel, int threads, size_t smem, std::atomic<int>* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const int r = sms * per_sm;
+  if (dev >= 0 && dev < 64 && r > 0) cache[dev].store(r, std::memory_order_relaxed);
+  return r;
+}
+
 template <int D, int HPC>
 static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t st) {
   using L = AttnLayout<D, HPC>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
   static std::atomic<uint64_t> configured{0};  // devices with the shared-memory limit raised
+  static std::atomic<int> resident[64];        // per device; zero-initialised (static storage)
   const cudaError_t e = ensure_dynamic_smem(prefill_attention_kernel<D, HPC>, L::kAlloc, configured);
   if (e != cudaSuccess) return e;
+  AttnParams q = p;
+  q.light_qtiles = p.n_qtiles;
+  if (p.heavy_by_head) {
+    const int r = resident_ctas(prefill_attention_kernel<D, HPC>, AttnRoles<HPC>::kThreads, L::kAlloc, resident);
+    q.light_qtiles = light_qtiles_for(p.n_qtiles, (long long)p.B * p.Hkv * p.n_groups, r);
+  }
   const unsigned grid = (unsigned)p.n_qtiles * p.B * p.Hkv * p.n_groups;
   return launch_dependent(prefill_attention_kernel<D, HPC>, dim3(grid), dim3(AttnRoles<HPC>::kThreads), L::kAlloc,
-                          st, tq, tk, tv, to, p);
+                          st, tq, tk, tv, to, q);
 }
 
 cudaError_t launch_prefill_attention(const AttnParams& p, int D, int hpc, const CUtensorMap& tq,
