@@ -62,6 +62,38 @@ def test_prefill_sweep(case):
     assert_close(lse, ref_lse, atol=LSE_ATOL, rel_l2=np.inf, what="lse")
 
 
+WORK_ORDER = [
+    # B, S, Hq, Hkv, D, spans: causal layers whose grid has both parts of the work order
+    (2, 4000, 16, 8, 128, [[100, 356], [2000, 2256]]),   # two-head CTAs, 16 units, ragged last tile
+    (1, 6100, 16, 4, 64, None),                          # two-head CTAs, G = 4: two head groups per kv head
+    (1, 6100, 8, 2, 256, [[5000, 5256]]),                # one-head CTAs (head dim 256)
+]
+
+
+@pytest.mark.parametrize("case", WORK_ORDER, ids=[f"B{c[0]}_S{c[1]}_H{c[2]}x{c[3]}_D{c[4]}" for c in WORK_ORDER])
+def test_causal_work_order_heavy_and_light_tiles(case):
+    """On a causal layer the heavy query tiles of each (sequence, kv head, head
+    group) unit run unit by unit and the light tiles of all units follow.
+    These shapes have more query tiles per unit than the light tail holds on
+    this GPU (at most one CTA per SM for these kernels, so the tail is at most
+    sqrt(2 * tiles * SMs / units) tiles), so both parts run; every row of every
+    head is compared."""
+    B, S, Hq, Hkv, D, spans = case
+    G = Hq // Hkv
+    units = B * Hkv * (G // 2 if D <= 128 else G)
+    nq = (S + 127) // 128
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert np.sqrt(2.0 * nq * sms / units) < nq - 2, "the case must reach the heavy part of the order"
+    xc = inputs.prefill_layer_inputs(B, S, Hq, Hkv, D, seed=11, layer=5)
+    xc["spans"] = _spans_tensor(spans, B)
+    xd = to_dev(xc)
+    out, lse = run_prefill(xd, GLB, 1024, 1e6, 8.0)
+    assert g3.check_device_error(g3.workspace(0, dev())) == 0
+    ref, ref_lse = oracle_rows(xc, GLB, 1024, 1e6, 8.0)
+    assert_close(out, ref)
+    assert_close(lse, ref_lse, atol=LSE_ATOL, rel_l2=np.inf, what="lse")
+
+
 def test_prefill_positions_shifted():
     """Shifting every position by a constant leaves the output unchanged."""
     B, S, Hq, Hkv, D = 1, 600, 4, 2, 128
