@@ -70,7 +70,7 @@ def launches_in_timed_region(trace: dict, steps: int, untraced_per_step: int = 0
     return (per_step + untraced_per_step) * steps
 
 
-def kernel_source_hash(files=("prefill.cu", "sm100_ptx.cuh", "g3_internal.h")) -> str:
+def kernel_source_hash(files=("prefill.cu", "sm100_ptx.cuh", "tmem_wide.cuh", "g3_internal.h")) -> str:
     """Hash of the sources a committed ncu traffic figure was taken on."""
     h = hashlib.sha256()
     for f in files:
