@@ -14,8 +14,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "prologue.cu", "prefill.cu", "decode.cu", "decode_static.cu", "projector.cu", "backward.cu"]
-HEADERS = ["g3_internal.h", "sm100_ptx.cuh", "tmem_wide.cuh", "func_attr.cuh", os.path.join("..", "..", "include", "g3attn.h")]
+SOURCES = ["api.cu", "prologue.cu", "prefill.cu", "decode.cu", "decode_static.cu", "projector.cu", "backward.cu", "backward256.cu"]
+HEADERS = ["g3_internal.h", "sm100_ptx.cuh", "tmem_wide.cuh", "func_attr.cuh", "backward_common.cuh", os.path.join("..", "..", "include", "g3attn.h")]
 LIB = os.path.join(HERE, "libg3attn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2",

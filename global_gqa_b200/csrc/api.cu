@@ -100,12 +100,12 @@ EncodeTiledFn encode_fn() {
 
 // [B, S, H, D] bf16, boxes of 64 features x 1 head x 128 tokens x 1 sequence,
 // 128-byte swizzle (matches the tcgen05 shared-memory descriptors).
-bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int D, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -588,8 +588,7 @@ g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v, c
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv))
     return fail(G3_ERR_INVALID_ARG, "prefill backward: bf16 tensors must be 16-byte aligned");
-  if (D != 64 && D != 128)
-    return fail(G3_ERR_UNSUPPORTED, "prefill backward: head_dim %d not built (64, 128)", D);
+  if (!supported_d(D)) return fail(G3_ERR_UNSUPPORTED, "prefill backward: head_dim %d not built (64, 128, 256)", D);
   if ((size_t)B * S * Hq * D >= (1ull << 40)) return fail(G3_ERR_UNSUPPORTED, "prefill backward: problem too large");
   const int G = Hq / Hkv;
   const long long n_qtiles = (S + g3::kTileRows - 1) / g3::kTileRows;
@@ -687,10 +686,24 @@ g3_status g3attn_prefill_backward(const void* q, const void* k, const void* v, c
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "prefill backward prologue: %s", cudaGetErrorString(e));
   e = traced("backward_prep", st, [&] { return g3::launch_bwd_prep(bp, D, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward prep: %s", cudaGetErrorString(e));
-  e = traced("backward_dkdv", st, [&] { return g3::launch_bwd_dkdv(bp, D, tq, tdo, tk, tv, st); });
-  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dk/dv: %s", cudaGetErrorString(e));
-  e = traced("backward_dq", st, [&] { return g3::launch_bwd_dq(bp, D, tq, tdo, tk, tv, st); });
-  if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dq: %s", cudaGetErrorString(e));
+  if (D == 256) {
+    // Head dim 256: 64-row sub-tiles on the streamed side, dV and dK from two kernels.
+    CUtensorMap tq64, tdo64, tk64, tv64;
+    if (!make_bshd_map(&tq64, pp.q_hat, B, S, Hq, D, 64) || !make_bshd_map(&tdo64, dout, B, S, Hq, D, 64) ||
+        !make_bshd_map(&tk64, pp.k_hat, B, S, Hkv, D, 64) || !make_bshd_map(&tv64, v, B, S, Hkv, D, 64))
+      return fail(G3_ERR_CUDA, "prefill backward: cuTensorMapEncodeTiled unavailable or failed");
+    e = traced("backward_dv", st, [&] { return g3::launch_bwd_dv256(bp, tq64, tdo64, tk, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dv: %s", cudaGetErrorString(e));
+    e = traced("backward_dk", st, [&] { return g3::launch_bwd_dk256(bp, tq64, tdo64, tk, tv, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dk: %s", cudaGetErrorString(e));
+    e = traced("backward_dq", st, [&] { return g3::launch_bwd_dq256(bp, tq, tdo, tk64, tv64, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dq: %s", cudaGetErrorString(e));
+  } else {
+    e = traced("backward_dkdv", st, [&] { return g3::launch_bwd_dkdv(bp, D, tq, tdo, tk, tv, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dk/dv: %s", cudaGetErrorString(e));
+    e = traced("backward_dq", st, [&] { return g3::launch_bwd_dq(bp, D, tq, tdo, tk, tv, st); });
+    if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward dq: %s", cudaGetErrorString(e));
+  }
   e = traced("backward_norm_rope", st, [&] { return g3::launch_bwd_norm_rope(bp, D, st); });
   if (e != cudaSuccess) return fail(G3_ERR_CUDA, "backward norm/rope: %s", cudaGetErrorString(e));
   return G3_OK;

@@ -40,6 +40,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "backward_common.cuh"
 #include "func_attr.cuh"
 #include "g3_internal.h"
 #include "sm100_ptx.cuh"
@@ -170,6 +171,7 @@ cudaError_t launch_bwd_prep(const BwdParams& p, int D, cudaStream_t st) {
   switch (D) {
     case 64: bwd_prep_kernel<64><<<(unsigned)blocks, kPrepThreads, 0, st>>>(p); break;
     case 128: bwd_prep_kernel<128><<<(unsigned)blocks, kPrepThreads, 0, st>>>(p); break;
+    case 256: bwd_prep_kernel<256><<<(unsigned)blocks, kPrepThreads, 0, st>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -359,6 +361,7 @@ cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st) {
   switch (D) {
     case 64: bwd_norm_rope_kernel<64><<<p.n_norm_blocks, kNormThreads, 0, st>>>(p); break;
     case 128: bwd_norm_rope_kernel<128><<<p.n_norm_blocks, kNormThreads, 0, st>>>(p); break;
+    case 256: bwd_norm_rope_kernel<256><<<p.n_norm_blocks, kNormThreads, 0, st>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaGetLastError();
@@ -368,23 +371,9 @@ cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st) {
 }
 
 // ================================================================ bwd_dkdv
-// Warp roles of both backward attention kernels: warp 0 TMA producer, warp 1
-// tensor-memory owner and tcgen05.mma issuer, warps 2-17 the elementwise work.
-// The elementwise step needs no row reduction (lse and delta are known), so
-// the 128 columns of a tile are split between two warps: four warps per TMEM
-// lane quarter, each on 16 rows x 64 columns; thread t holds rows t/4 and
-// t/4+8 of its slice and columns 64h + 8k + 2(t%4) + {0,1}, k < 8, of its half h.
-constexpr int kBwdEwWarps = 16;
-constexpr int kBwdThreads = (2 + kBwdEwWarps) * 32;
-constexpr int kBwdEwThreads = kBwdEwWarps * 32;
-constexpr int kBwdFirstWarp = 2;
-
-// Elementwise warp e = warp - 2: TMEM lane quarter warp % 4 (hardware rule),
-// 16-row half (e >> 2) & 1, column half e >> 3.
-__device__ __forceinline__ int bwd_lane_base(int warp) {
-  return (warp & 3) * 32 + (((warp - kBwdFirstWarp) >> 2) & 1) * 16;
-}
-__device__ __forceinline__ int bwd_col_half(int warp) { return (warp - kBwdFirstWarp) >> 3; }
+// The thread layout (backward_common.cuh) with 128-column tiles: each warp
+// covers 16 rows x 64 columns; thread t holds columns 64h + 8k + 2(t%4) +
+// {0,1}, k < 8, of its half h.
 
 // The bf16 tile a column half packs (P^T, dS^T, dS) goes over the first 32 of
 // its own 64 fp32 columns, so no warp overwrites columns another warp has yet
@@ -398,7 +387,6 @@ __device__ __forceinline__ void tmem_ld_half(uint32_t taddr, float* v) {
   if constexpr (D == 128) tmem_ld_16x256b_x8(taddr, v);
   else tmem_ld_16x256b_x4(taddr, v);
 }
-constexpr int kBwdSwizzleBlock = 128 * 64 * 2;  // 128 rows x 64 bf16
 
 constexpr int kBwdMaxStages = 4;
 struct BwdBarriers {

@@ -170,6 +170,14 @@ cudaError_t launch_bwd_dkdv(const BwdParams& p, int D, const CUtensorMap& tm_q, 
 cudaError_t launch_bwd_dq(const BwdParams& p, int D, const CUtensorMap& tm_q, const CUtensorMap& tm_do,
                           const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
 cudaError_t launch_bwd_norm_rope(const BwdParams& p, int D, cudaStream_t st);
+// Head dim 256 (backward256.cu): maps with 64-row boxes for the streamed
+// sub-tiles, 128-row boxes for the resident tiles.
+cudaError_t launch_bwd_dv256(const BwdParams& p, const CUtensorMap& tm_q64, const CUtensorMap& tm_do64,
+                             const CUtensorMap& tm_k, cudaStream_t st);
+cudaError_t launch_bwd_dk256(const BwdParams& p, const CUtensorMap& tm_q64, const CUtensorMap& tm_do64,
+                             const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t st);
+cudaError_t launch_bwd_dq256(const BwdParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_do,
+                             const CUtensorMap& tm_k64, const CUtensorMap& tm_v64, cudaStream_t st);
 
 cudaError_t launch_decode_prologue(const DecodeParams& p, int D, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeParams& p, int D, int grid_chunks, cudaStream_t st);

@@ -175,8 +175,7 @@ size_t g3attn_prefill_backward_workspace_size(int32_t B, int32_t S, int32_t Hq, 
  *   q, k, v, q_gamma, k_gamma, positions, layer_kind, window, rope_base,
  *   interp_factor, image_spans, n_spans, B, S, Hq, Hkv
  *              exactly as given to the forward g3attn_prefill call
- *   D          in {64, 128} (head_dim 256 is not built for the backward:
- *              G3_ERR_UNSUPPORTED)
+ *   D          in {64, 128, 256} (G3_ERR_UNSUPPORTED otherwise)
  *   out        bf16 [B, S, Hq, D]  the forward call's output
  *   lse        fp32 [B, Hq, S]     the forward call's lse (required)
  *   dout       bf16 [B, S, Hq, D]  gradient of the loss with respect to out

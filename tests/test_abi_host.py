@@ -138,7 +138,7 @@ def _backward(lib, **kw):
     (dict(lse=None), 1), (dict(dout=None), 1), (dict(dq=None), 1), (dict(dk_gamma=None, dkg=None), 1),
     (dict(B=0), 1), (dict(Hq=3), 1), (dict(kind=5), 1), (dict(window=0), 1), (dict(interp=float("nan")), 1),
     (dict(n_spans=1), 1), (dict(dv=FAKE + 8), 1), (dict(dout=FAKE + 2), 1),
-    (dict(D=256), 2), (dict(D=96), 2), (dict(ws=None), 3), (dict(ws=FAKE * 256 + 64), 3), (dict(wsb=4096), 3),
+    (dict(D=512), 2), (dict(D=96), 2), (dict(ws=None), 3), (dict(ws=FAKE * 256 + 64), 3), (dict(wsb=4096), 3),
 ])
 def test_prefill_backward_rejects_on_host(lib, kw, code):
     kw.pop("dk_gamma", None)
