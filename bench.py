@@ -409,6 +409,7 @@ def run_gpu(args, rank, world, local_rank):
               if v is not None}
         out1 = torch.empty_like(x1["q"])
         ws1 = torch.empty(g3.prefill_workspace_size(1, S1, Hq1, Hkv1, D1), dtype=torch.uint8, device=dev)
+        bws1 = torch.empty(g3.prefill_backward_workspace_size(1, S1, Hq1, Hkv1, D1), dtype=torch.uint8, device=dev)
         shapes_1b = {"workload": "B1 S32768 Hq4 Hkv1 D256 (Gemma 3 1B shapes)"}
         for kind, W, base, interp, name in ((0, 1024, 1e4, 1.0, "local"), (1, S1, 1e6, 8.0, "global")):
             f = metrics.layer_flops(1, S1, Hq1, D1, kind, W)
@@ -428,7 +429,42 @@ def run_gpu(args, rank, world, local_rank):
             npro, mpro = tr.get("prefill_prologue", (1, 0.0))
             shapes_1b[name] = {"flops": f, "attention_us": 1e3 * ma / na,
                                "attention_tflops": f / (ma / na * 1e-3) / 1e12, "prologue_us": 1e3 * mpro / npro}
-        del x1, out1, ws1
+            # The backward of the same layer, from its out / lse and a random dout.
+            o1, l1 = g3.prefill(x1["q"], x1["k"], x1["v"], x1["q_gamma"], x1["k_gamma"], x1["positions"], kind, W,
+                                base, interp, return_lse=True, ws=ws1, stream=stream)
+            do1 = torch.empty_like(o1)
+            inputs.device_fill_normal_bf16(do1, seed=200 + kind)
+            g1 = {"dq": torch.empty_like(x1["q"]), "dk": torch.empty_like(x1["k"]), "dv": torch.empty_like(x1["v"]),
+                  "dq_gamma": torch.empty(D1, dtype=torch.float32, device=dev),
+                  "dk_gamma": torch.empty(D1, dtype=torch.float32, device=dev)}
+
+            def backward_1b():
+                g3.prefill_backward(x1["q"], x1["k"], x1["v"], x1["q_gamma"], x1["k_gamma"], x1["positions"], kind,
+                                    W, base, interp, None, o1, l1, do1, grads=g1, ws=bws1, stream=stream)
+
+            for _ in range(2):
+                backward_1b()
+            if g3.check_device_error(bws1) != 0:
+                raise RuntimeError("device error in the head-dim-256 backward warm-up")
+            g3.trace_collect()
+            barrier()
+            g3.trace_enable(True)
+            e0g = torch.cuda.Event(enable_timing=True)
+            e1g = torch.cuda.Event(enable_timing=True)
+            e0g.record(stream)
+            for _ in range(3):
+                backward_1b()
+            e1g.record(stream)
+            barrier()
+            g3.trace_enable(False)
+            tr = g3.trace_collect()
+            bms = e0g.elapsed_time(e1g) / 3
+            shapes_1b[name]["backward"] = {
+                "ms": bms, "tflops_algorithmic": 2.5 * f / (bms * 1e-3) / 1e12,
+                "kernels_us": {k: 1e3 * m / n for k, (n, m) in tr.items() if n > 0},
+                "note": "dV, dK and dQ kernels of head dim 256 (64-row streamed sub-tiles); trace on every call"}
+            del o1, l1, do1, g1
+        del x1, out1, ws1, bws1
 
     # ---- image soft tokens (outside the timed region): 64 images, 64x64 patch
     # grid of 1152 features each, 4x4 pool -> 256 tokens; HBM-bound
