@@ -36,6 +36,13 @@ METRIC = "prefill attn TFLOP/s (unmasked FLOPs, 5:1 block) & decode KV GB/s, 1 B
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "prefill_attention_traffic.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 data-sheet figures (dense bf16, HBM3e), reported beside the measured peaks.
+NOMINAL = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+
+
+def fractions(value: float, measured: float, nominal: float) -> dict:
+    """A block-level rate as a fraction of the measured peak and of the data-sheet peak."""
+    return {"of_measured": value / measured if measured else None, "of_nominal": value / nominal}
 
 
 def peaks():
@@ -333,7 +340,8 @@ def run_gpu(args, rank, world, local_rank):
         pass
     peak_tf = pk["bf16_tflops"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": (achieved / peak_tf) if achieved else None, "traffic": traffic,
+                "frac": (achieved / peak_tf) if achieved else None,
+                "frac_of_nominal": (achieved / NOMINAL["bf16_tflops"]) if achieved else None, "traffic": traffic,
                 "kernel": "prefill_attention", "peak_kind": f"{pk_kind} dense bf16 burst",
                 "launches": n_attn, "avg_launch_ms": attn_ms / max(n_attn, 1),
                 "traced_steps": n_traced(args.steps)}
@@ -654,6 +662,7 @@ def run_gpu(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": block_config(cfg, world, block_flops),
+        "value_frac": fractions(value / max(world, 1), peak_tf, NOMINAL["bf16_tflops"]),
         "roofline": roofline,
         "kernels": kernels,
         "layer_kinds": layer_kinds,
@@ -739,8 +748,10 @@ def run_decode(args, dev, stream, rank, world, pk, pk_kind):
                    "kv_bytes_per_step": all_bytes, "l2": "inputs larger than L2 (~38 GB of cache read per step)",
                    "parallelism": f"batch split by sequence over {world} rank(s)", "sequences_per_rank": B},
         "scaling": "strong",
+        "value_frac": fractions(gbs / max(world, 1), pk["hbm_gbs"], NOMINAL["hbm_gbs"]),
         "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": (ach / pk["hbm_gbs"]) if ach else None,
+                     "frac_of_nominal": (ach / NOMINAL["hbm_gbs"]) if ach else None,
                      "traffic": decode_traffic_per_launch(step_bytes / len(blk)), "kernel": "decode_split",
                      "peak_kind": f"{pk_kind} copy bandwidth", "launches": n_split,
                      "traced_steps": n_traced(args.steps)},
@@ -862,11 +873,14 @@ def run_long_blocks(args, dev, stream, rank, world, pk, pk_kind):
                        "parallelism": f"kv heads split over {world} rank(s)", "kv_heads_per_rank": cfg.Hkv},
             "scaling": "strong",
             "ms_per_block": ms, "tflops": flops_all / (ms * 1e-3) / 1e12, "blocks_timed": reps,
+            "value_frac": fractions(flops_all / (ms * 1e-3) / 1e12 / max(world, 1), pk["bf16_tflops_sustained"],
+                                    NOMINAL["bf16_tflops"]),
             # Blocks of 27-180 ms run for seconds back to back: the GPU settles at
             # its power-capped clock, so the peak is the sustained matmul figure.
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": (ach / pk["bf16_tflops_sustained"]) if ach else None,
-                         "frac_of_burst": (ach / pk["bf16_tflops"]) if ach else None, "traffic": None,
+                         "frac_of_burst": (ach / pk["bf16_tflops"]) if ach else None,
+                         "frac_of_nominal": (ach / NOMINAL["bf16_tflops"]) if ach else None, "traffic": None,
                          "kernel": "prefill_attention",
                          "peak_kind": f"{pk_kind} dense bf16 sustained (seconds-long, under the power cap)",
                          "launches": n_attn, "avg_launch_ms": attn_ms / max(n_attn, 1)},

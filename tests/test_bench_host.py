@@ -57,3 +57,10 @@ def test_long_block_spans_are_the_workloads():
     assert (sp[:, 1:, 0] >= sp[:, :-1, 1]).all() and sp.min() >= 0 and sp.max() <= cfg.S
     assert np.array_equal(sp, bench.long_block_spans(cfg).numpy())
     assert bench.long_block_spans(inputs.LONG_128K) is None
+
+
+def test_fractions_of_measured_and_nominal_peaks():
+    f = bench.fractions(750.0, 1618.8, bench.NOMINAL["bf16_tflops"])
+    assert abs(f["of_measured"] - 750.0 / 1618.8) < 1e-12
+    assert abs(f["of_nominal"] - 750.0 / 2250.0) < 1e-12
+    assert bench.fractions(1.0, 0.0, 2.0)["of_measured"] is None
