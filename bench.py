@@ -234,9 +234,9 @@ def decode_traffic_per_launch(alg_bytes_per_launch: float):
     return None
 
 
-def oracle_extras_baselines(line: dict) -> None:
-    """The oracles of the backward and of the soft tokens, timed as they stand
-    on bounded samples of the same workloads (rank 0, N = 1)."""
+def oracle_extras_baselines(line: dict, budget_s: float) -> None:
+    """The oracles of the backward, of decode and of the soft tokens, timed as
+    they stand on bounded samples of the same workloads (rank 0, N = 1)."""
     from oracle import backward as BW
     from oracle import projector as PJ
     cfg = inputs.BLOCK_8K
@@ -255,6 +255,35 @@ def oracle_extras_baselines(line: dict) -> None:
             "seconds": secs, "sample": f"gradients of kv head 0 and its {G} query heads over the first {S1} tokens "
                                        f"of a local layer (W={L.window}) of {cfg.name} (algorithmic FLOPs), "
                                        f"float64 numpy"}
+    if line.get("decode"):
+        # One local (ring) and the global layer of the first sequences of the
+        # 64-sequence batch, until about half the budget is spent.
+        from oracle import attention as OA
+        dc = inputs.DECODE_B64
+        blk = dc.block()
+        lens = inputs.decode_lengths(dc.B, dc.len_lo, dc.len_hi, dc.seed)
+        nbytes, secs, n_seq = 0, 0.0, 0
+        for b in range(dc.B):
+            for li in (0, len(blk) - 1):
+                L = blk[li]
+                Lb = int(lens[b])
+                n_hist = (Lb - 1) if L.kind == 1 else min(Lb, L.window) - 1
+                hist = inputs.cache_history(n_hist, dc.Hkv, dc.D, seed=dc.seed, layer=li, batch=b)
+                st = inputs.decode_step_inputs(1, dc.Hq, dc.Hkv, dc.D, seed=dc.seed, layer=li)
+                t0 = time.perf_counter()
+                OA.decode(st["q"], st["k_new"], st["v_new"], st["q_gamma"], st["k_gamma"], np.array([Lb]),
+                          [hist["k"]], [hist["v"]], np.array([Lb - 1 - n_hist]), L.kind, L.window, L.rope_base,
+                          L.interp)
+                secs += time.perf_counter() - t0
+                nbytes += metrics.decode_kv_bytes([Lb], dc.Hkv, dc.D, L.kind, L.window)
+            n_seq += 1
+            if secs > budget_s / 2:
+                break
+        line["decode"]["cpu_baseline"] = {
+            "value": nbytes / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "seconds": secs, "sample": f"the first {n_seq} of the {dc.B} sequences of {dc.name}, one ring layer "
+                                       f"and the global layer each (KV bytes counted as the GPU metric counts "
+                                       f"them), float64 numpy"}
     if line.get("soft_tokens"):
         Bi, gh, F = 8, 64, 1152
         px = np.random.default_rng(17).standard_normal((Bi, gh * gh, F)).astype(np.float32)
@@ -1031,7 +1060,7 @@ def main():
                                 "sample": f"{r} query rows (groups of 64 per layer, all 32 heads) of the "
                                           f"{inputs.BLOCK_8K.name} block, float64 numpy"}
         if args.extras and args.cpu_budget > 0:
-            oracle_extras_baselines(line)
+            oracle_extras_baselines(line, args.cpu_budget)
             oracle_long_baselines(line.get("long_blocks"), args.cpu_budget / 2)
     if rank == 0:
         print(json.dumps(line), flush=True)
