@@ -218,7 +218,6 @@ def test_backward_1b_shapes_32k_closed_form(kind):
     want = x["dout"].double().sum(dim=(1, 2))  # [B, D]
     have = got["dv"].double().sum(dim=(1, 2)).cpu()
     rel = (have - want).norm() / want.norm()
-    print(f"1B shapes, kind {kind}: closed-form relative error {rel:.3e}")
     assert rel < 1e-2, rel
     for name in ("dq", "dk", "dq_gamma", "dk_gamma"):
         assert torch.isfinite(got[name].float()).all(), name
