@@ -59,10 +59,11 @@ DECODE_TRAFFIC_PATH = os.path.join(ROOT, "profiles", "decode_split_traffic.json"
 
 # The library's per-kernel trace brackets each launch with CUDA events; an event
 # between two kernels keeps the next launch from starting until the previous one
-# has drained (~5 us per kernel boundary, ~4 % of the 8K block step).  So the
-# timed loops carry the trace on every TRACE_EVERY-th step only (the first one
-# included), and a kernel's average duration comes from those steps' launches.
-TRACE_EVERY = 4
+# has drained (~5.7 us per kernel boundary, ~4 % of a traced 8K block step).  So
+# the timed loops carry the trace on every TRACE_EVERY-th step only (the first
+# one included: two of the default 20 steps), and a kernel's average duration
+# comes from those steps' launches.
+TRACE_EVERY = 10
 
 
 def n_traced(steps: int) -> int:
