@@ -134,14 +134,14 @@ def test_8k_block_sampled_rows():
 def test_mixed_32k_sampled_rows():
     def rows(c, x):
         sp = x["spans"][0].numpy()
-        r = sampled_rows(c.S, 1024, sp, n_random=256)
+        r = sampled_rows(c.S, 1024, sp, n_random=1024)
         return r
     _block_parity(inputs.MIXED_32K, rows, layers=[0, 5])
 
 
 @pytest.mark.parametrize("layer", [0, 5])
 def test_long_128k_sampled_rows(layer):
-    _block_parity(inputs.LONG_128K, lambda c, x: sampled_rows(c.S, 1024, n_random=64), layers=[layer])
+    _block_parity(inputs.LONG_128K, lambda c, x: sampled_rows(c.S, 1024, n_random=1024), layers=[layer])
 
 
 # -------------------------------------------------------------- cache fill
